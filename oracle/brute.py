@@ -1,0 +1,146 @@
+"""Literal-loop MLA for tiny shapes.  TEST INFRASTRUCTURE ONLY.
+
+Pure Python (lists and the math module, no numpy arithmetic) so that it shares
+no vectorised code with oracle/mla_ref.py; tests use it to pin the oracle on
+shapes of a few elements. Same readings as mla_ref (see its docstrings):
+eps inside the root, interleaved pairs (2i, 2i+1), scale 1/sqrt(d_n + d_r),
+per-head [k_nope | v] columns of wkv_b, cache row [latent | k_pe] or
+[k_pe | latent].
+"""
+from __future__ import annotations
+
+import math
+
+
+def _mat(a):
+    return [[float(v) for v in row] for row in a]
+
+
+def _vecmat(v, m):
+    """v [K] times m [K][N] -> [N]."""
+    K, N = len(m), len(m[0])
+    return [sum(v[k] * m[k][j] for k in range(K)) for j in range(N)]
+
+
+def _rms(v, g, eps):
+    ms = sum(x * x for x in v) / len(v)
+    r = 1.0 / math.sqrt(ms + eps)
+    return [v[i] * r * g[i] for i in range(len(v))]
+
+
+def _rope(v, pos, theta):
+    d = len(v)
+    out = list(v)
+    for i in range(d // 2):
+        phi = pos * theta ** (-2.0 * i / d)
+        a, b = v[2 * i], v[2 * i + 1]
+        out[2 * i] = a * math.cos(phi) - b * math.sin(phi)
+        out[2 * i + 1] = a * math.sin(phi) + b * math.cos(phi)
+    return out
+
+
+def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens,
+                slot_mapping, layout=0):
+    """One whole decode step, loops only.
+
+    cache_rows: list of flat cache rows (lists of R floats), mutated copy returned.
+    Returns (out [n][hidden], head_out [n][H][d_v], q_abs [n][H][r_kv],
+    q_pe [n][H][d_r], new cache_rows).
+    """
+    H, dn, dr, dv = cfg.n_heads, cfg.qk_nope, cfg.qk_rope, cfg.v_dim
+    rkv, bs = cfg.kv_lora_rank, cfg.block_size
+    wkv_b = _mat(W["wkv_b"])
+    rows = [list(r) for r in cache_rows]
+    q_abs_all, q_pe_all = [], []
+    for t, x in enumerate(hidden):
+        x = [float(v) for v in x]
+        pos = int(positions[t])
+        if cfg.q_lora_rank:
+            ql = _rms(_vecmat(x, _mat(W["wq_a"])), [float(g) for g in W["q_norm_w"]], cfg.norm_eps)
+            q = _vecmat(ql, _mat(W["wq_b"]))
+        else:
+            q = _vecmat(x, _mat(W["wq_b"]))
+        kv = _vecmat(x, _mat(W["wkv_a"]))
+        c = _rms(kv[:rkv], [float(g) for g in W["kv_norm_w"]], cfg.norm_eps)
+        kpe = _rope(kv[rkv:], pos, cfg.rope_theta)
+        q_abs_t, q_pe_t = [], []
+        for h in range(H):
+            qh = q[h * (dn + dr):(h + 1) * (dn + dr)]
+            qn, qp = qh[:dn], _rope(qh[dn:], pos, cfg.rope_theta)
+            # absorption through the nope columns of head h of wkv_b
+            qa = [sum(qn[p] * wkv_b[cc][h * (dn + dv) + p] for p in range(dn)) for cc in range(rkv)]
+            q_abs_t.append(qa)
+            q_pe_t.append(qp)
+        q_abs_all.append(q_abs_t)
+        q_pe_all.append(q_pe_t)
+        slot = int(slot_mapping[t])
+        if slot >= 0:
+            rows[slot] = (c + kpe) if layout == 0 else (kpe + c)
+    scale = 1.0 / math.sqrt(dn + dr)
+    head_out = []
+    for t in range(len(hidden)):
+        L = int(context_lens[t])
+        ctx = []
+        for j in range(L):
+            r = rows[int(block_table[t][j // bs]) * bs + j % bs]
+            ctx.append((r[:rkv], r[rkv:]) if layout == 0 else (r[dr:], r[:dr]))
+        o_t = []
+        for h in range(H):
+            s = [(sum(q_abs_all[t][h][cc] * ctx[j][0][cc] for cc in range(rkv))
+                  + sum(q_pe_all[t][h][i] * ctx[j][1][i] for i in range(dr))) * scale
+                 for j in range(L)]
+            mx = max(s)
+            e = [math.exp(v - mx) for v in s]
+            z = sum(e)
+            o_lat = [sum(e[j] / z * ctx[j][0][cc] for j in range(L)) for cc in range(rkv)]
+            o_t.append([sum(o_lat[cc] * wkv_b[cc][h * (dn + dv) + dn + d] for cc in range(rkv))
+                        for d in range(dv)])
+        head_out.append(o_t)
+    wo = _mat(W["wo"])
+    out = [_vecmat([v for h in range(H) for v in head_out[t][h]], wo) for t in range(len(hidden))]
+    return out, head_out, q_abs_all, q_pe_all, rows
+
+
+def prefill(cfg, W, hidden):
+    """Causal expanded prefill of one sequence at positions 0..S-1, loops only.
+    Returns (out [S][hidden], head_out [S][H][d_v])."""
+    H, dn, dr, dv = cfg.n_heads, cfg.qk_nope, cfg.qk_rope, cfg.v_dim
+    rkv = cfg.kv_lora_rank
+    S = len(hidden)
+    wkv_b = _mat(W["wkv_b"])
+    Q, K, V = [], [], []
+    for i, x in enumerate(hidden):
+        x = [float(v) for v in x]
+        if cfg.q_lora_rank:
+            ql = _rms(_vecmat(x, _mat(W["wq_a"])), [float(g) for g in W["q_norm_w"]], cfg.norm_eps)
+            q = _vecmat(ql, _mat(W["wq_b"]))
+        else:
+            q = _vecmat(x, _mat(W["wq_b"]))
+        kv = _vecmat(x, _mat(W["wkv_a"]))
+        c = _rms(kv[:rkv], [float(g) for g in W["kv_norm_w"]], cfg.norm_eps)
+        kpe = _rope(kv[rkv:], i, cfg.rope_theta)
+        kvo = _vecmat(c, wkv_b)
+        Qi, Ki, Vi = [], [], []
+        for h in range(H):
+            qh = q[h * (dn + dr):(h + 1) * (dn + dr)]
+            Qi.append(qh[:dn] + _rope(qh[dn:], i, cfg.rope_theta))
+            base = h * (dn + dv)
+            Ki.append(kvo[base:base + dn] + kpe)
+            Vi.append(kvo[base + dn:base + dn + dv])
+        Q.append(Qi)
+        K.append(Ki)
+        V.append(Vi)
+    scale = 1.0 / math.sqrt(dn + dr)
+    head_out = []
+    for i in range(S):
+        o_i = []
+        for h in range(H):
+            s = [sum(Q[i][h][d] * K[j][h][d] for d in range(dn + dr)) * scale for j in range(i + 1)]
+            mx = max(s)
+            e = [math.exp(v - mx) for v in s]
+            z = sum(e)
+            o_i.append([sum(e[j] / z * V[j][h][d] for j in range(i + 1)) for d in range(dv)])
+        head_out.append(o_i)
+    wo = _mat(W["wo"])
+    out = [_vecmat([v for h in range(H) for v in head_out[i][h]], wo) for i in range(S)]
+    return out, head_out
