@@ -1,0 +1,44 @@
+// Host-side state of one MLA layer: configuration, the repacked weight blob's
+// layout, and what the tensor-core path prepares at init.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+#include "tc_state.cuh"
+
+static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+static inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// Launches of this library's kernels (mla_kernel_launch_count).
+void mla_count_launch(int k);
+
+// Repacked weight blob.
+// Every matrix is stored K-major, [N, K] (the transpose of the pages' [in,
+// out] form), so that one output feature's weights are contiguous:
+//   W1   [Nq1 + R, D]   rows [0, Nq1) = wq_a^T (or q_proj^T), then wkv_a^T
+//   Wqb  [H*(d_n+d_r), r_q]                          (r_q > 0)
+//   Wuk  [H][r_kv][d_n]   Wuk[h][c][p] = wkv_b[c][h*(d_n+d_v) + p]
+//   Wuv  [H][d_v][r_kv]   Wuv[h][d][c] = wkv_b[c][h*(d_n+d_v) + d_n + d]
+//   Wkvb [H*(d_n+d_v), r_kv]                          (prefill)
+//   Wo   [D, H*d_v]
+// FP8 blobs add fp32 scales per 128x128 block of each K-major matrix,
+// [ceil(N/128)][ceil(K/128)].
+struct WeightLayout {
+  int Nq1, N1, R, Hq, Hkv;
+  size_t esz;
+  size_t W1, Wqb, Wuk, Wuv, Wkvb, Wo, gq, gkv;
+  size_t sW1, sWqb, sWuk, sWuv, sWkvb, sWo;
+  size_t total;
+};
+
+struct mla_handle {
+  mla_config cfg;
+  WeightLayout L;
+  float scale;
+  char* base;
+  int device;
+  TcState tc;
+};
+

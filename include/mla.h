@@ -1,0 +1,241 @@
+/*
+ * mla.h -- C-ABI of a B200 (sm_100a) implementation of one DeepSeek-style
+ * Multi-head Latent Attention (MLA) layer step: the decode front-fold, the
+ * absorbed decode attention over a paged latent cache, and the expanded
+ * causal prefill.
+ *
+ * Conventions shared by every entry point
+ *   - Every call returns int: MLA_OK (0) or a negative MLA_ERR_* code;
+ *     mla_strerror() names it. On an error return nothing was launched.
+ *   - Pointers named "device" must be device memory on the current device;
+ *     "host" pointers are host memory. All device work is enqueued,
+ *     asynchronously, on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - The library never allocates device memory. The caller owns every
+ *     buffer: weights blob, workspace, KV cache, inputs and outputs.
+ *     mla_init_weights() allocates one small host-side handle.
+ *   - Matrices are row-major. Weights are given in [in, out] form (y = x @ W),
+ *     as the pages give them ("MLA Decode QKV Kernel API Reference",
+ *     Parameters; "QKV CTE MLA Kernel API Reference", qkv_mla_mx parameters).
+ *   - Activation dtype (MLA_F32 or MLA_BF16) applies to hidden states,
+ *     q_abs / q_pe, the KV cache, head_out and out. RoPE tables and RMSNorm
+ *     gammas are always fp32.
+ *   - Content errors that only the device can see (a slot or block id out of
+ *     range, a context length out of range) set bits of a sticky int32 flag in
+ *     the workspace; the offending write or row is skipped. Read the flag with
+ *     mla_read_device_flag() and clear it with mla_clear_device_flag().
+ *
+ * Notation: n tokens, H heads, hidden D, q_lora_rank r_q, kv_lora_rank r_kv,
+ * qk_nope d_n, qk_rope d_r, v_dim d_v, R = r_kv + d_r (cache row width).
+ */
+#ifndef MLA_B200_MLA_H_
+#define MLA_B200_MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define MLA_OK 0
+#define MLA_ERR_INVALID_ARG (-1)   /* bad pointer, size, shape or enum value */
+#define MLA_ERR_UNSUPPORTED (-2)   /* valid request this build does not implement */
+#define MLA_ERR_CUDA (-3)          /* a CUDA runtime call or launch failed */
+#define MLA_ERR_DEVICE_FLAG (-4)   /* the device flag is non-zero (see below) */
+#define MLA_ERR_WORKSPACE (-5)     /* workspace / weights buffer too small */
+
+/* Device flag bits (sticky, OR-ed by kernels). */
+#define MLA_FLAG_BAD_SLOT 1        /* slot_mapping[t] >= n_blocks * block_size */
+#define MLA_FLAG_BAD_BLOCK 2       /* block_table entry outside [0, n_blocks) */
+#define MLA_FLAG_BAD_CONTEXT 4     /* context_lens[t] < 1 or > max_context_len */
+#define MLA_FLAG_WAIT_TIMEOUT 8    /* a bounded device-side wait gave up */
+
+/* ---- configuration ----------------------------------------------------- */
+typedef enum {
+  MLA_F32 = 0,
+  MLA_BF16 = 1,
+  /* FP8-E4M3 (OCP) codes, one byte per weight, with fp32 scales per 128x128
+   * block: W[k][n] = e4m3(code[k][n]) * scale[k/128][n/128], scale tensor
+   * [ceil(in/128), ceil(out/128)] row-major. "Struct MlaWeights", field
+   * wq_a_fp8 (128x128 block scales, dequantised in fp32 before the MAC with
+   * bf16 activations); scale shape as "QKV CTE MLA Kernel API Reference",
+   * *_scale_hbm. Weights only; needs act_dtype MLA_BF16. */
+  MLA_FP8_E4M3_B128 = 2
+} mla_dtype;
+
+typedef enum {
+  /* cache row = [latent (r_kv) | k_pe (d_r)], DeepSeek's order */
+  MLA_ROW_LATENT_FIRST = 0,
+  /* cache row = [k_pe (d_r) | latent (r_kv)], the inverted order of
+   * "MLA Decode QKV Kernel API Reference", Notes */
+  MLA_ROW_PE_FIRST = 1
+} mla_row_layout;
+
+/* Layer shape ("struct Mla" fields; "MLA Decode QKV Kernel API Reference",
+ * Dimensions). Limits of this build: d_r even; r_kv, d_n, d_v, d_r, D and
+ * H*(d_n+d_r) multiples of 8 (16-byte rows); for MLA_FP8_E4M3_B128 also
+ * r_q, d_n, d_v, H*(d_n+d_r) multiples of 128. */
+typedef struct {
+  int hidden;          /* D */
+  int n_heads;         /* H */
+  int q_lora_rank;     /* r_q; 0 = one full query projection x @ q_proj */
+  int kv_lora_rank;    /* r_kv */
+  int qk_nope;         /* d_n: per-head query/key dims RoPE does not rotate */
+  int qk_rope;         /* d_r: per-head dims RoPE rotates (the trailing ones) */
+  int v_dim;           /* d_v */
+  int block_size;      /* rows per paged-cache block */
+  float norm_eps;      /* RMSNorm epsilon ("... norm_eps", default 1e-6) */
+  float softmax_scale; /* 0 => 1/sqrt(d_n + d_r) ("struct Mla", field scale) */
+  int act_dtype;       /* mla_dtype: MLA_F32 or MLA_BF16 */
+  int weight_dtype;    /* mla_dtype: must equal act_dtype, or MLA_FP8_E4M3_B128 */
+  int row_layout;      /* mla_row_layout */
+} mla_config;
+
+/* Weights in [in, out] row-major form, device pointers, element type
+ * weight_dtype (uint8 codes for FP8). Only read during mla_init_weights().
+ *   wq_a  [D, r_q]                  (NULL when q_lora_rank == 0)
+ *   wq_b  [r_q, H*(d_n+d_r)]        or, when q_lora_rank == 0, the full
+ *                                   q_proj [D, H*(d_n+d_r)]
+ *   wkv_a [D, r_kv + d_r]           output order [latent | k_pe]
+ *   wkv_b [r_kv, H*(d_n+d_v)]       per head [k_nope_h | v_h] columns
+ *   wo    [H*d_v, D]
+ *   q_norm_w [r_q] fp32 (NULL when q_lora_rank == 0), kv_norm_w [r_kv] fp32
+ *   *_scale: FP8 only, fp32 [ceil(in/128), ceil(out/128)], else NULL. */
+typedef struct {
+  const void* wq_a;
+  const void* wq_b;
+  const void* wkv_a;
+  const void* wkv_b;
+  const void* wo;
+  const float* q_norm_w;
+  const float* kv_norm_w;
+  const float* wq_a_scale;
+  const float* wq_b_scale;
+  const float* wkv_a_scale;
+  const float* wkv_b_scale;
+  const float* wo_scale;
+} mla_weights_desc;
+
+typedef struct mla_handle mla_handle;
+
+/* ---- weights ------------------------------------------------------------ */
+
+/* Bytes of the library's repacked weight blob for `cfg` (0 if cfg is invalid). */
+size_t mla_weights_bytes(const mla_config* cfg);
+
+/* Validate cfg, repack the weights into `dst` (device, >= mla_weights_bytes,
+ * 256-byte aligned, owned by the caller and kept alive while the handle is
+ * used), enqueue the repack on `stream`, and return a host handle in *out.
+ * The repack merges [wq_a | wkv_a] into one first projection ("Struct
+ * MlaWeights", wkv_a_merged; "QKV CTE MLA Kernel API Reference", Combined Q/KV
+ * Path Stage 1) and slices wkv_b into W_UK [H, d_n, r_kv] and W_UV
+ * [H, r_kv, d_v] ("Struct MlaWeights", w_uk_t and w_uv). The source weights
+ * may be freed once the stream has passed the repack. */
+int mla_init_weights(const mla_config* cfg, const mla_weights_desc* w, void* dst,
+                     size_t dst_bytes, void* stream, mla_handle** out);
+
+/* Release the host handle (not `dst`). NULL is ignored. */
+void mla_destroy(mla_handle* h);
+
+/* ---- workspace ------------------------------------------------------------ */
+
+/* Bytes of device workspace the calls below need for up to `max_tokens`
+ * decode tokens (or prefill sequence length) and contexts of up to
+ * `max_context_len` rows. */
+size_t mla_workspace_bytes(const mla_handle* h, int max_tokens, int max_context_len);
+
+/* Zero the workspace (device flag and internal counters). Call once on a new
+ * workspace before its first use; the library keeps it consistent afterwards. */
+int mla_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Copy the device flag to *flag_out (synchronises `stream`). Returns
+ * MLA_ERR_DEVICE_FLAG when it is non-zero, MLA_OK otherwise. */
+int mla_read_device_flag(const void* ws, int* flag_out, void* stream);
+int mla_clear_device_flag(void* ws, void* stream);
+
+/* ---- RoPE tables ---------------------------------------------------------- */
+
+/* cos/sin [n, d_r/2] fp32 (device) of positions[n] (device int32):
+ * angle_i = pos * theta^(-2i/d_r), evaluated in fp64 on the device and
+ * rounded once to fp32. Half width as "MLA Decode QKV Kernel API Reference",
+ * Parameters (cos, sin: [n_tokens, qk_rope_dim // 2]). */
+int mla_rope_cos_sin(const int32_t* positions, int n, int qk_rope, double theta,
+                     float* cos_out, float* sin_out, void* stream);
+
+/* ---- decode ----------------------------------------------------------------- */
+
+/* The decode front-fold ("MLA Decode QKV Kernel API Reference",
+ * mla_decode_qkv): for each of n tokens (one per sequence)
+ *   q_lat = x @ wq_a; q = rms_norm(q_lat, q_norm_w) @ wq_b  (or x @ q_proj)
+ *   q_pe  = RoPE(q[h, d_n:]) per head, interleaved pairs (2i, 2i+1)
+ *   q_abs[h] = q[h, :d_n] @ W_UK[h]
+ *   kv = x @ wkv_a; c = rms_norm(kv[:r_kv], kv_norm_w); k_pe = RoPE(kv[r_kv:])
+ *   kv_cache row slot_mapping[t] = [c | k_pe] (or [k_pe | c], per row_layout)
+ * hidden      device [n, D] act dtype
+ * cos, sin    device [n, d_r/2] fp32, the token's position (mla_rope_cos_sin)
+ * kv_cache    device [n_blocks, 1, block_size, R] act dtype, mutated in place
+ * slot_mapping device [n] int32 flat row (block * block_size + offset);
+ *             negative = skip the token's write; >= n_blocks*block_size sets
+ *             MLA_FLAG_BAD_SLOT and skips. Slots must be distinct.
+ * q_abs       device [n, H, r_kv] act dtype (output)
+ * q_pe        device [n, H, d_r] act dtype (output)
+ * input_norm_w must be NULL (a folded input RMSNorm is not implemented).
+ * ws          device workspace (mla_workspace_bytes with max_tokens >= n). */
+int mla_decode_qkv(mla_handle* h, const void* hidden, int n, const float* cos,
+                   const float* sin, void* kv_cache, int n_blocks,
+                   const int32_t* slot_mapping, void* q_abs, void* q_pe,
+                   const float* input_norm_w, void* ws, size_t ws_bytes, void* stream);
+
+/* Absorbed decode attention, V extraction and o_proj ("Struct MlaWeights",
+ * w_uk_t / w_uv / wo; "struct Mla", scale): for token t (sequence t) with
+ * L = context_lens[t] cached rows at positions 0..L-1,
+ *   s[h, j] = (q_abs[h] . c_j + q_pe[h] . k_pe_j) * softmax_scale
+ *   o_lat[h] = softmax_j(s[h]) @ c;  head_out[h] = o_lat[h] @ W_UV[h]
+ *   out = concat_h(head_out[h]) @ wo
+ * Row j of sequence t is flat cache row block_table[t][j / bs] * bs + j % bs.
+ * q_abs, q_pe    device, as written by mla_decode_qkv
+ * kv_cache       device [n_blocks, 1, bs, R] act dtype (read only)
+ * block_table    device [n, max_blocks_per_seq] int32
+ * context_lens   device [n] int32, 1 <= L <= max_context_len (includes this
+ *                step's token, which mla_decode_qkv wrote at position L-1)
+ * max_context_len host int, an upper bound on every context_lens[t]
+ * out            device [n, D] act dtype
+ * head_out       device [n, H, d_v] act dtype, or NULL
+ * Must follow mla_decode_qkv on the same stream when both are used for one
+ * step (the scatter writes the row attention reads). */
+int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe,
+                    const void* kv_cache, int n_blocks, const int32_t* block_table,
+                    int max_blocks_per_seq, const int32_t* context_lens,
+                    int max_context_len, int n, void* out, void* head_out, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* ---- prefill ------------------------------------------------------------------ */
+
+/* Causal prefill (context encoding) of one sequence of S tokens at positions
+ * 0..S-1 with K/V expanded from the latent ("QKV CTE MLA Kernel API
+ * Reference", qkv_mla_mx: Stage 1 x @ [wq_a | wkv_a]; Q Stage 2; KV Stage 2
+ * norm(kv) @ wkv_b split into k_nope, v; RoPE on q_pe and k_pe, k_pe
+ * broadcast to every head), then softmax(Q K^T * scale) V with query i seeing
+ * keys j <= i, and o_proj.
+ * hidden   device [S, D] act dtype; cos, sin device [S, d_r/2] fp32
+ * out      device [S, D] act dtype; head_out device [S, H, d_v] or NULL
+ * kv_cache / slot_mapping: optional (both NULL or both set): the sequence's
+ *          cache rows are scattered as in mla_decode_qkv. */
+int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos,
+                const float* sin, void* out, void* head_out, void* kv_cache,
+                int n_blocks, const int32_t* slot_mapping, void* ws, size_t ws_bytes,
+                void* stream);
+
+/* ---- misc ------------------------------------------------------------------------ */
+
+const char* mla_strerror(int status);
+
+/* Launches of the library's own kernels since load (all entry points). */
+uint64_t mla_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_MLA_H_ */
