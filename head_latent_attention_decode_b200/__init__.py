@@ -35,7 +35,7 @@ SYMBOLS = (
     "mla_weights_bytes", "mla_init_weights", "mla_destroy", "mla_workspace_bytes",
     "mla_workspace_init", "mla_read_device_flag", "mla_clear_device_flag", "mla_rope_cos_sin",
     "mla_decode_qkv", "mla_decode_attn", "mla_prefill", "mla_strerror",
-    "mla_kernel_launch_count",
+    "mla_kernel_launch_count", "mla_set_kernel_timer",
 )
 
 
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.mla_strerror.argtypes = [i]
         L.mla_kernel_launch_count.restype = ctypes.c_uint64
         L.mla_kernel_launch_count.argtypes = []
+        L.mla_set_kernel_timer.restype = i
+        L.mla_set_kernel_timer.argtypes = [ctypes.c_char_p, vp, vp]
         _lib = L
     return _lib
 
@@ -213,3 +215,13 @@ def mla_prefill(handle, hidden, cos, sin, out, ws, head_out=None, kv_cache=None,
 
 def mla_kernel_launch_count() -> int:
     return int(lib().mla_kernel_launch_count())
+
+
+def mla_set_kernel_timer(kernel: str | None, start=None, stop=None) -> None:
+    """Bracket every launch of `kernel` with records of two torch.cuda.Event
+    (enable_timing=True); None clears the timer."""
+    if kernel is None:
+        _check(lib().mla_set_kernel_timer(None, None, None), "mla_set_kernel_timer")
+        return
+    _check(lib().mla_set_kernel_timer(kernel.encode(), start.cuda_event, stop.cuda_event),
+           "mla_set_kernel_timer")

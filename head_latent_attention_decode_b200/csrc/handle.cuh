@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cuda_runtime.h>
+
 #include "../../include/mla.h"
 #include "tc_state.cuh"
 
@@ -13,6 +15,10 @@ static inline long long cdiv(long long a, long long b) { return (a + b - 1) / b;
 
 // Launches of this library's kernels (mla_kernel_launch_count).
 void mla_count_launch(int k);
+
+// Kernel timer (mla_set_kernel_timer): bracket a launch with event records.
+void mla_timer_begin(const char* kernel, cudaStream_t s);
+void mla_timer_end(const char* kernel, cudaStream_t s);
 
 // Repacked weight blob.
 // Every matrix is stored K-major, [N, K] (the transpose of the pages' [in,

@@ -18,6 +18,22 @@ static std::atomic<unsigned long long> g_launches{0};
 void mla_count_launch(int k) { g_launches.fetch_add((unsigned long long)k); }
 static inline void count_launch(int k = 1) { mla_count_launch(k); }
 
+static char g_timer_kernel[32] = {0};
+static cudaEvent_t g_timer_start = nullptr, g_timer_stop = nullptr;
+
+static void timer_record(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  else cudaEventRecord(ev, s);
+}
+void mla_timer_begin(const char* k, cudaStream_t s) {
+  if (g_timer_kernel[0] && strcmp(k, g_timer_kernel) == 0) timer_record(g_timer_start, s);
+}
+void mla_timer_end(const char* k, cudaStream_t s) {
+  if (g_timer_kernel[0] && strcmp(k, g_timer_kernel) == 0) timer_record(g_timer_stop, s);
+}
+
 
 static int validate_config(const mla_config* c) {
   if (!c) return MLA_ERR_INVALID_ARG;
@@ -206,6 +222,15 @@ const char* mla_strerror(int s) {
 }
 
 uint64_t mla_kernel_launch_count(void) { return (uint64_t)g_launches.load(); }
+
+int mla_set_kernel_timer(const char* kernel, void* start_event, void* stop_event) {
+  if (!kernel) { g_timer_kernel[0] = 0; g_timer_start = g_timer_stop = nullptr; return MLA_OK; }
+  if (!start_event || !stop_event || strlen(kernel) >= sizeof(g_timer_kernel)) return MLA_ERR_INVALID_ARG;
+  strcpy(g_timer_kernel, kernel);
+  g_timer_start = (cudaEvent_t)start_event;
+  g_timer_stop = (cudaEvent_t)stop_event;
+  return MLA_OK;
+}
 
 size_t mla_weights_bytes(const mla_config* cfg) {
   if (validate_config(cfg) != MLA_OK) return 0;
@@ -412,8 +437,10 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
   const int R = rkv + dr;
   const size_t smem = (size_t)(ATT_TR * (R + 1) + ATT_HPB * R) * 4;
   dim3 grid(W.splits, n, (unsigned)cdiv(H, ATT_HPB));
+  mla_timer_begin("attn", s);
   if (ta == 0) { set_smem(attn_decode_simt_kernel<float>, smem); attn_decode_simt_kernel<float><<<grid, 256, smem, s>>>(p); }
   else { set_smem(attn_decode_simt_kernel<bf16>, smem); attn_decode_simt_kernel<bf16><<<grid, 256, smem, s>>>(p); }
+  mla_timer_end("attn", s);
   count_launch();
   void* o_lat = wsb + W.o_lat;
   dim3 cg(n, H);
@@ -493,8 +520,10 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos, cons
   pa.scale = h->scale;
   const size_t smem = (size_t)(PA_BQ * (dn + dr) + PA_BK * (dn + dr + 1) + PA_BK * dv) * 4;
   dim3 grid((unsigned)cdiv(S, PA_BQ), H);
+  mla_timer_begin("prefill_attn", s);
   if (ta == 0) { set_smem(prefill_attn_simt_kernel<float>, smem); prefill_attn_simt_kernel<float><<<grid, 128, smem, s>>>(pa); }
   else { set_smem(prefill_attn_simt_kernel<bf16>, smem); prefill_attn_simt_kernel<bf16><<<grid, 128, smem, s>>>(pa); }
+  mla_timer_end("prefill_attn", s);
   count_launch();
   launch_linear(ta, tw, ta, lin(head, (long long)H * dv, h->base + L.Wo, (long long)H * dv, wscale(h, L.sWo),
                                 cdiv((long long)H * dv, 128), out, D, S, D, H * dv), 1, s);

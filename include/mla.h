@@ -234,6 +234,15 @@ const char* mla_strerror(int status);
 /* Launches of the library's own kernels since load (all entry points). */
 uint64_t mla_kernel_launch_count(void);
 
+/* Kernel timer (tracing). While set, every launch of the library kernel named
+ * `kernel` (one of "attn", "front", "gemm", "prefill_attn"; NULL clears the
+ * timer) is bracketed by records of the two events (cudaEvent_t, created by
+ * the caller with timing enabled) on the launch stream, so that
+ * cudaEventElapsedTime(start, stop) is that kernel's device time. Inside a
+ * stream capture the records become external event-record nodes of the graph.
+ * Process-wide; not thread-safe against concurrent launches. */
+int mla_set_kernel_timer(const char* kernel, void* start_event, void* stop_event);
+
 #ifdef __cplusplus
 }
 #endif

@@ -129,7 +129,8 @@ def test_scatter_touches_only_mapped_rows_bit_exact():
     cos, sin = ref.rope_cos_sin(case.inp.positions, s.qk_rope, s.rope_theta)
     c, k_pe = ref.kv_projection(s, W, case.inp.hidden, cos, sin)
     rows = ref.cache_row(c, k_pe, ref.LATENT_FIRST)
-    got = cache.reshape(n_rows, -1).cpu().numpy().astype(np.float64)
+    with np.errstate(invalid="ignore"):             # sentinel rows may hold NaN patterns
+        got = cache.reshape(n_rows, -1).cpu().numpy().astype(np.float64)
     for t, slot in enumerate(slots):
         if slot >= 0:
             assert_close(got[slot], rows[t], TOL["f32"], f"row {slot}")
