@@ -305,6 +305,9 @@ def kernel_time(step, kernel, k, flush, stream):
     """Average device ms of one library kernel inside the step (graph with event
     nodes around that kernel's launch)."""
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)          # torch creates the CUDA events on first record
+    b.record(stream)
+    torch.cuda.synchronize()
     mla.mla_set_kernel_timer(kernel, a, b)
     try:
         g = torch.cuda.CUDAGraph()

@@ -424,7 +424,9 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
   void* head = head_out ? head_out : (void*)(wsb + W.head);
   if (tc_decode_attn_supported(h, n, max_context_len)) {
     const int r = tc_decode_attn(h, q_abs, q_pe, kv_cache, n_blocks, block_table, max_blocks_per_seq,
-                                 context_lens, max_context_len, n, out, head, wsb, W.tc, s);
+                                 context_lens, max_context_len, n, out, head, wsb, W.tc, s,
+                                 (float*)(wsb + W.part_o), (float*)(wsb + W.part_ml), W.splits,
+                                 (bf16*)(wsb + W.o_lat));
     return r != MLA_OK ? r : cuda_status();
   }
   AttnArgs p{};
@@ -478,7 +480,7 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos, cons
   void* head = head_out ? head_out : (void*)(wsb + W.phead);
   if (tc_prefill_supported(h, S)) {
     const int r = tc_prefill(h, hidden, S, cos, sin, out, head, kv_cache, n_blocks, slot_mapping, wsb,
-                             W.pY1, s);
+                             W.pY1, W.pqn, W.pQ, W.pcn, W.pkpe, W.pKV, s);
     return r != MLA_OK ? r : cuda_status();
   }
   float* Y1 = (float*)(wsb + W.pY1);

@@ -1,0 +1,313 @@
+// Persistent, warp-specialised tcgen05 GEMM for the layer's weight contractions:
+//   D[b][m][n] = sum_k A[b][m][k] * B[b][n][k]      (bf16 in, fp32 accumulate)
+// A and B are K-major and arrive by TMA (128-byte swizzle) into a STAGES-deep
+// shared-memory ring; one thread issues tcgen05.mma (M = 128, N = BN, K = 16)
+// into one of two TMEM accumulators; four epilogue warps drain the other
+// accumulator (tcgen05.ld) while the next tile accumulates. Work units are
+// (m tile, n tile, batch, K split), taken round-robin by a grid of at most one
+// CTA per SM.
+//
+// Decode uses it "swap-AB": A = weights (M = output features), B = the few
+// tokens (N = tokens), so that no tensor-core row is padding; prefill uses it
+// with A = tokens. The epilogue modes write fp32 split partials, bf16 rows, or
+// the query with interleaved RoPE applied to its q_pe columns.
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace mla {
+namespace tc {
+
+enum EpiMode : int {
+  EPI_F32_T = 0,    // out_f32[(split*N + n)*ldo + m]                  (A = weights)
+  EPI_BF16_T = 1,   // out_bf16[n*ldo + b*bstride + m]
+  EPI_QROPE_T = 2,  // m = h*(dn+dr)+j, n = token: j < dn -> out_bf16 q_nope[n][h][j];
+                    //   else RoPE pair -> out2_bf16 q_pe[n][h][j-dn]
+  EPI_BF16_N = 3,   // out_bf16[m*ldo + b*bstride + n]                 (A = tokens)
+  EPI_F32_N = 4,    // out_f32[(split*M + m)*ldo + n]
+  EPI_QROPE_N = 5,  // m = token, n = h*(dn+dr)+j: out_bf16[m*ldo + n], q_pe columns rotated
+};
+
+struct GemmArgs {
+  int M, N, K;
+  int m_tiles, n_tiles, batches, splits, kb_per_split, k_blocks, total_units;
+  int a_rows_dim2, b_rows_dim2;   // tensor-map dim holding the rows: 0 -> dim 1, 1 -> dim 2
+  int mode;
+  void* out;
+  long long ldo, bstride;
+  void* out2;
+  const float* cos;
+  const float* sin;
+  int H, dn, dr;
+  int* flag;
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;   // two accumulators
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int SMEM = 1024 + BAR_OFF + 256;
+};
+
+__device__ __forceinline__ void gemm_store(const GemmArgs& g, int m, int n0, int split, int b, const uint32_t* r) {
+  const bool m_ok = m < g.M;
+  switch (g.mode) {
+    case EPI_F32_T: {
+      if (!m_ok) break;
+      float* o = (float*)g.out;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int n = n0 + j;
+        if (n < g.N) o[((long long)split * g.N + n) * g.ldo + m] = __uint_as_float(r[j]);
+      }
+      break;
+    }
+    case EPI_BF16_T: {
+      if (!m_ok) break;
+      bf16* o = (bf16*)g.out;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int n = n0 + j;
+        if (n < g.N) o[(long long)n * g.ldo + (long long)b * g.bstride + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+      }
+      break;
+    }
+    case EPI_QROPE_T: {
+      const int hd = g.dn + g.dr;
+      const int h = m / hd, jj = m % hd;
+      const bool odd = (m & 1) != 0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float v = __uint_as_float(r[j]);
+        const float partner = __shfl_xor_sync(0xffffffffu, v, 1);   // all lanes take part
+        const int n = n0 + j;
+        if (!m_ok || n >= g.N) continue;
+        if (jj < g.dn) {
+          ((bf16*)g.out)[((long long)n * g.H + h) * g.dn + jj] = __float2bfloat16_rn(v);
+        } else {
+          const int i = (jj - g.dn) >> 1;
+          const float c = g.cos[(long long)n * (g.dr >> 1) + i], s = g.sin[(long long)n * (g.dr >> 1) + i];
+          const float o = odd ? (partner * s + v * c) : (v * c - partner * s);
+          ((bf16*)g.out2)[((long long)n * g.H + h) * g.dr + (jj - g.dn)] = __float2bfloat16_rn(o);
+        }
+      }
+      break;
+    }
+    case EPI_BF16_N: {
+      if (!m_ok) break;
+      bf16* o = (bf16*)g.out + (long long)m * g.ldo + (long long)b * g.bstride;
+      if (n0 + 16 <= g.N && ((((uintptr_t)(o + n0)) & 15) == 0)) {
+        uint4 v0, v1;
+        v0.x = pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1]));
+        v0.y = pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3]));
+        v0.z = pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5]));
+        v0.w = pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7]));
+        v1.x = pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9]));
+        v1.y = pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11]));
+        v1.z = pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13]));
+        v1.w = pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15]));
+        *reinterpret_cast<uint4*>(o + n0) = v0;
+        *reinterpret_cast<uint4*>(o + n0 + 8) = v1;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (n0 + j < g.N) o[n0 + j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+      }
+      break;
+    }
+    case EPI_F32_N: {
+      if (!m_ok) break;
+      float* o = (float*)g.out + ((long long)split * g.M + m) * g.ldo;
+      if (n0 + 16 <= g.N && ((((uintptr_t)(o + n0)) & 15) == 0)) {
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(o + n0 + j) =
+              make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                          __uint_as_float(r[j + 3]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (n0 + j < g.N) o[n0 + j] = __uint_as_float(r[j]);
+      }
+      break;
+    }
+    case EPI_QROPE_N: {
+      if (!m_ok) break;
+      const int hd = g.dn + g.dr;
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+#pragma unroll
+      for (int j = 0; j < 16; j += 2) {
+        const int jj = (n0 + j) % hd;      // n0 + j even, so (jj, jj+1) is one RoPE pair
+        if (jj >= g.dn) {
+          const int i = (jj - g.dn) >> 1;
+          const float c = g.cos[(long long)m * (g.dr >> 1) + i], s = g.sin[(long long)m * (g.dr >> 1) + i];
+          const float a = v[j], bb = v[j + 1];
+          v[j] = a * c - bb * s;
+          v[j + 1] = a * s + bb * c;
+        }
+      }
+      bf16* o = (bf16*)g.out + (long long)m * g.ldo;
+      if (n0 + 16 <= g.N && ((((uintptr_t)(o + n0)) & 15) == 0)) {
+        uint4 v0, v1;
+        v0.x = pack_bf16x2(v[0], v[1]); v0.y = pack_bf16x2(v[2], v[3]);
+        v0.z = pack_bf16x2(v[4], v[5]); v0.w = pack_bf16x2(v[6], v[7]);
+        v1.x = pack_bf16x2(v[8], v[9]); v1.y = pack_bf16x2(v[10], v[11]);
+        v1.z = pack_bf16x2(v[12], v[13]); v1.w = pack_bf16x2(v[14], v[15]);
+        *reinterpret_cast<uint4*>(o + n0) = v0;
+        *reinterpret_cast<uint4*>(o + n0 + 8) = v1;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (n0 + j < g.N) o[n0 + j] = __float2bfloat16_rn(v[j]);
+      }
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+__device__ __forceinline__ void decode_unit(const GemmArgs& g, int u, int& mt, int& nt, int& b, int& s) {
+  mt = u % g.m_tiles;
+  u /= g.m_tiles;
+  nt = u % g.n_tiles;
+  u /= g.n_tiles;
+  b = u % g.batches;
+  s = u / g.batches;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t a_base = sbase;                                  // [STAGES][A]
+  const uint32_t b_base = sbase + C::STAGES * C::A_BYTES;          // [STAGES][B]
+  const uint32_t bar = sbase + C::BAR_OFF;
+  auto full_bar = [&](int s) { return bar + 8 * s; };
+  auto empty_bar = [&](int s) { return bar + 8 * (C::STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar + 8 * (2 * C::STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar + 8 * (2 * C::STAGES + 2 + a); };
+  const uint32_t final_bar = bar + 8 * (2 * C::STAGES + 4);
+  uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + 8 * (2 * C::STAGES + 5));
+  volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 128); }
+    mbar_init(final_bar, 1);
+    *abort_word = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
+  if (warp == 0) { tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
+        int mt, nt, b, s;
+        decode_unit(g, u, mt, nt, b, s);
+        const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % C::STAGES, round = it / C::STAGES;
+          if (!mbar_wait(empty_bar(st), (round & 1) ^ 1, abort_word, g.flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(st), C::STAGE_BYTES);
+          const int ar = mt * C::BM, br = nt * BN;
+          if (g.a_rows_dim2) tma_load_3d(a_base + st * C::A_BYTES, &tmA, full_bar(st), kb * C::BK, b, ar);
+          else tma_load_3d(a_base + st * C::A_BYTES, &tmA, full_bar(st), kb * C::BK, ar, b);
+          if (g.b_rows_dim2) tma_load_3d(b_base + st * C::B_BYTES, &tmB, full_bar(st), kb * C::BK, b, br);
+          else tma_load_3d(b_base + st * C::B_BYTES, &tmB, full_bar(st), kb * C::BK, br, b);
+        }
+      }
+      // drain: every load issued has landed before the CTA can exit
+      const int first = it > C::STAGES ? it - C::STAGES : 0;
+      for (int j = first; j < it; ++j) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(full_bar(j % C::STAGES), (j / C::STAGES) & 1)) {
+          if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(g.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, BN);
+      int it = 0, tile = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x, ++tile) {
+        int mt, nt, b, s;
+        decode_unit(g, u, mt, nt, b, s);
+        const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
+        const int acc = tile & 1, use = tile >> 1;
+        if (!mbar_wait(tempty_bar(acc), (use & 1) ^ 1, abort_word, g.flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % C::STAGES, round = it / C::STAGES;
+          if (!mbar_wait(full_bar(st), round & 1, abort_word, g.flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = a_base + st * C::A_BYTES, sb = b_base + st * C::B_BYTES;
+#pragma unroll
+          for (int k = 0; k < C::BK / 16; ++k)
+            mma_bf16(d, sdesc_sw128(sa + 32 * k), sdesc_sw128(sb + 32 * k), idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          mma_commit(empty_bar(st));
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar(acc));
+      }
+      // all MMAs complete before teardown
+      mma_commit(final_bar);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(final_bar, 0)) {
+        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(g.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
+      }
+    }
+  } else {
+    // ---------------- epilogue: warps 0..3 <-> TMEM lanes 32w..32w+31 ----------------
+    int tile = 0;
+    for (int u = blockIdx.x; u < g.total_units; u += gridDim.x, ++tile) {
+      int mt, nt, b, s;
+      decode_unit(g, u, mt, nt, b, s);
+      const int acc = tile & 1, use = tile >> 1;
+      if (!mbar_wait(tfull_bar(acc), use & 1, abort_word, g.flag)) break;
+      tc_fence_after();
+      const int m = mt * C::BM + warp * 32 + lane;
+      const uint32_t row_addr = tmem + ((uint32_t)(warp * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(row_addr + c * 16, r);
+        tmem_ld_wait();
+        gemm_store(g, m, nt * BN + c * 16, s, b, r);
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace tc
+}  // namespace mla

@@ -1,17 +1,434 @@
 // Tensor-core (tcgen05 / TMEM / TMA) path of the MLA layer step for bf16
-// activations with bf16 or FP8 weights.
+// activations with bf16 weights: every weight contraction runs on the
+// persistent tcgen05 GEMM (tc_gemm.cuh); the norms, RoPE and the cache scatter
+// run in the GEMM epilogues or in one per-token front-fold kernel.
 #pragma once
 
-#include "handle.cuh"
+#include <cudaTypedefs.h>
 
-static inline size_t tc_decode_ws_bytes(const mla_handle*, long long, int) { return 0; }
-static inline int tc_init(mla_handle* h) { h->tc.enabled = 0; return MLA_OK; }
-static inline bool tc_decode_qkv_supported(const mla_handle*, int) { return false; }
-static inline bool tc_decode_attn_supported(const mla_handle*, int, int) { return false; }
-static inline bool tc_prefill_supported(const mla_handle*, int) { return false; }
-static inline int tc_decode_qkv(const mla_handle*, const void*, int, const float*, const float*, void*, int,
-                                const int32_t*, void*, void*, char*, size_t, cudaStream_t) { return MLA_ERR_UNSUPPORTED; }
-static inline int tc_decode_attn(const mla_handle*, const void*, const void*, const void*, int, const int32_t*,
-                                 int, const int32_t*, int, int, void*, void*, char*, size_t, cudaStream_t) { return MLA_ERR_UNSUPPORTED; }
-static inline int tc_prefill(const mla_handle*, const void*, int, const float*, const float*, void*, void*, void*,
-                             int, const int32_t*, char*, size_t, cudaStream_t) { return MLA_ERR_UNSUPPORTED; }
+#include "handle.cuh"
+#include "simt_kernels.cuh"
+#include "tc_gemm.cuh"
+
+namespace mla {
+namespace tc {
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (cuTensorMapEncodeTiled, resolved through the runtime so the
+// library needs no link-time libcuda)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }
+  return fn;
+}
+
+// bf16 3-D map {K, d1, d2} (K contiguous) with 128-byte swizzle and a box of
+// 64 K-elements x `box_rows` rows; the rows are dimension 1 (rows_dim2 = 0) or
+// dimension 2 (rows_dim2 = 1). Strides in bytes. Out-of-range elements read 0.
+static int make_map(CUtensorMap* m, const void* base, long long K, long long d1, long long d2, long long s1,
+                    long long s2, int box_rows, int rows_dim2) {
+  auto fn = encode_fn();
+  if (!fn) return MLA_ERR_CUDA;
+  if (((uintptr_t)base) & 15 || s1 % 16 || s2 % 16) return MLA_ERR_UNSUPPORTED;
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)d1, (cuuint64_t)d2};
+  cuuint64_t strides[2] = {(cuuint64_t)s1, (cuuint64_t)s2};
+  cuuint32_t box[3] = {64, (cuuint32_t)(rows_dim2 ? 1 : box_rows), (cuuint32_t)(rows_dim2 ? box_rows : 1)};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// 2-D row-major [rows, K] bf16 matrix with row stride ld (elements).
+static int make_map2(CUtensorMap* m, const void* base, long long K, long long rows, long long ld, int box_rows) {
+  return make_map(m, base, K, rows, 1, ld * 2, ld * 2 * rows, box_rows, 0);
+}
+
+template <int BN>
+static int launch_gemm_bn(const CUtensorMap& A, const CUtensorMap& B, const GemmArgs& g, int num_sms,
+                          cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    attr_set[dev] = true;
+  }
+  const int grid = g.total_units < num_sms ? g.total_units : num_sms;
+  tc_gemm_kernel<BN><<<grid, 192, C::SMEM, s>>>(A, B, g);
+  mla_count_launch(1);
+  return MLA_OK;
+}
+
+static int pick_bn(int n) {
+  if (n <= 16) return 16;
+  if (n <= 32) return 32;
+  if (n <= 64) return 64;
+  if (n <= 128) return 128;
+  return 256;
+}
+
+// Fill the tiling fields of g and launch with an N tile of `bn`.
+static int launch_gemm(const CUtensorMap& A, const CUtensorMap& B, GemmArgs g, int bn, int splits, int num_sms,
+                       cudaStream_t s) {
+  g.m_tiles = (int)cdiv(g.M, 128);
+  g.n_tiles = (int)cdiv(g.N, bn);
+  g.k_blocks = (int)cdiv(g.K, 64);
+  if (splits < 1) splits = 1;
+  if (splits > g.k_blocks) splits = g.k_blocks;
+  g.kb_per_split = (int)cdiv(g.k_blocks, splits);
+  g.splits = (int)cdiv(g.k_blocks, g.kb_per_split);   // no empty split
+  g.total_units = g.m_tiles * g.n_tiles * g.batches * g.splits;
+  if (g.total_units <= 0) return MLA_OK;
+  switch (bn) {
+    case 16: return launch_gemm_bn<16>(A, B, g, num_sms, s);
+    case 32: return launch_gemm_bn<32>(A, B, g, num_sms, s);
+    case 64: return launch_gemm_bn<64>(A, B, g, num_sms, s);
+    case 128: return launch_gemm_bn<128>(A, B, g, num_sms, s);
+    default: return launch_gemm_bn<256>(A, B, g, num_sms, s);
+  }
+}
+
+// Splits of the K loop so that (M tiles x splits) fills the SMs about twice.
+static int decode_splits_for(int m_tiles, int k_blocks, int num_sms) {
+  int s = (int)cdiv(2 * num_sms, m_tiles);
+  if (s > 16) s = 16;
+  if (s > k_blocks) s = k_blocks;
+  if (s < 1) s = 1;
+  // the launcher drops empty splits; report what it will use
+  const int per = (int)cdiv(k_blocks, s);
+  return (int)cdiv(k_blocks, per);
+}
+
+// ---------------------------------------------------------------------------
+// small kernels of the tensor-core decode path
+// ---------------------------------------------------------------------------
+struct FrontFoldTcArgs {
+  const float* Yp;  long long split_stride; int splits; int N1;
+  int rq, Nq1, rkv, dr, H, dn;
+  const float* q_norm_w; const float* kv_norm_w; float eps;
+  const float* cos; const float* sin;
+  bf16* qn; bf16* q_nope; bf16* q_pe;
+  bf16* cache; long long n_rows; const int* slot; int layout;
+  int* flag;
+};
+
+// One CTA per token: sum the K-split partials of x @ W1, then
+//   q latent -> RMSNorm * q_norm_w -> qn (bf16)                          (r_q > 0)
+//   or q -> q_nope (bf16) and RoPE(q_pe) (bf16)                          (r_q = 0)
+//   kv latent -> RMSNorm * kv_norm_w, k_pe -> RoPE, row -> cache[slot]
+__global__ void __launch_bounds__(256) frontfold_tc_kernel(FrontFoldTcArgs p) {
+  extern __shared__ float y[];   // [N1]
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  for (int c = threadIdx.x; c < p.N1; c += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < p.splits; ++s) acc += p.Yp[s * p.split_stride + (long long)t * p.N1 + c];
+    y[c] = acc;
+  }
+  __syncthreads();
+  const int half = p.dr / 2;
+  if (p.rq) {
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < p.rq; i += blockDim.x) ss += y[i] * y[i];
+    const float r = rsqrtf(block_sum(ss, red) / (float)p.rq + p.eps);
+    for (int i = threadIdx.x; i < p.rq; i += blockDim.x)
+      p.qn[(long long)t * p.rq + i] = __float2bfloat16_rn(y[i] * r * p.q_norm_w[i]);
+  } else {
+    const int hd = p.dn + p.dr;
+    for (int idx = threadIdx.x; idx < p.H * p.dn; idx += blockDim.x) {
+      const int h = idx / p.dn, j = idx % p.dn;
+      p.q_nope[(long long)t * p.H * p.dn + idx] = __float2bfloat16_rn(y[h * hd + j]);
+    }
+    for (int idx = threadIdx.x; idx < p.H * half; idx += blockDim.x) {
+      const int h = idx / half, i = idx % half;
+      float o0, o1;
+      rope_pair(y[h * hd + p.dn + 2 * i], y[h * hd + p.dn + 2 * i + 1], p.cos[(long long)t * half + i],
+                p.sin[(long long)t * half + i], &o0, &o1);
+      p.q_pe[((long long)t * p.H + h) * p.dr + 2 * i] = __float2bfloat16_rn(o0);
+      p.q_pe[((long long)t * p.H + h) * p.dr + 2 * i + 1] = __float2bfloat16_rn(o1);
+    }
+  }
+  const float* kv = y + p.Nq1;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < p.rkv; i += blockDim.x) ss += kv[i] * kv[i];
+  const float r = rsqrtf(block_sum(ss, red) / (float)p.rkv + p.eps);
+  const int slot = p.slot[t];
+  if (slot < 0) return;
+  if ((long long)slot >= p.n_rows) {
+    if (threadIdx.x == 0) set_flag(p.flag, MLA_FLAG_BAD_SLOT);
+    return;
+  }
+  bf16* row = p.cache + (long long)slot * (p.rkv + p.dr);
+  const int lat_off = (p.layout == MLA_ROW_LATENT_FIRST) ? 0 : p.dr;
+  const int pe_off = (p.layout == MLA_ROW_LATENT_FIRST) ? p.rkv : 0;
+  for (int i = threadIdx.x; i < p.rkv; i += blockDim.x)
+    row[lat_off + i] = __float2bfloat16_rn(kv[i] * r * p.kv_norm_w[i]);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    float o0, o1;
+    rope_pair(kv[p.rkv + 2 * i], kv[p.rkv + 2 * i + 1], p.cos[(long long)t * half + i],
+              p.sin[(long long)t * half + i], &o0, &o1);
+    row[pe_off + 2 * i] = __float2bfloat16_rn(o0);
+    row[pe_off + 2 * i + 1] = __float2bfloat16_rn(o1);
+  }
+}
+
+// out[n][m] = bf16(sum_s part[s][n][m])
+__global__ void splitk_reduce_bf16_kernel(const float* part, int splits, long long count, bf16* out) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
+       i += (long long)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < splits; ++s) acc += part[s * count + i];
+    out[i] = __float2bfloat16_rn(acc);
+  }
+}
+
+}  // namespace tc
+}  // namespace mla
+
+// ---------------------------------------------------------------------------
+// entry points used by mla_abi.cu
+// ---------------------------------------------------------------------------
+using namespace mla;
+using namespace mla::tc;
+
+struct TcDecodeWs {
+  size_t Yp, qn, q_nope, wo_part, total;
+  int s1, s5;
+};
+
+static TcDecodeWs tc_decode_ws(const mla_handle* h, long long n) {
+  TcDecodeWs w{};
+  const mla_config& c = h->cfg;
+  const WeightLayout& L = h->L;
+  const int sms = h->tc.num_sms > 0 ? h->tc.num_sms : 148;
+  w.s1 = decode_splits_for((int)cdiv(L.N1, 128), (int)cdiv(c.hidden, 64), sms);
+  w.s5 = decode_splits_for((int)cdiv(c.hidden, 128), (int)cdiv((long long)c.n_heads * c.v_dim, 64), sms);
+  size_t off = 0;
+  auto put = [&](size_t b) { size_t o = off; off = align_up(off + b, 256); return o; };
+  w.Yp = put((size_t)w.s1 * n * L.N1 * 4);
+  w.qn = put((size_t)n * (c.q_lora_rank ? c.q_lora_rank : 8) * 2);
+  w.q_nope = put((size_t)n * c.n_heads * c.qk_nope * 2);
+  w.wo_part = put((size_t)w.s5 * n * c.hidden * 4);
+  w.total = off;
+  return w;
+}
+
+static inline size_t tc_decode_ws_bytes(const mla_handle* h, long long n, int) {
+  if (!h->tc.enabled) return 0;
+  return tc_decode_ws(h, n).total;
+}
+
+static inline int tc_init(mla_handle* h) {
+  TcState& T = h->tc;
+  T.enabled = 0;
+  int dev = 0, major = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&T.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  const mla_config& c = h->cfg;
+  if (major != 10 || c.act_dtype != MLA_BF16 || c.weight_dtype != MLA_BF16) return MLA_OK;
+  if (c.hidden % 64 || c.kv_lora_rank % 64 || c.qk_nope % 64 || c.q_lora_rank % 64 ||
+      ((long long)c.n_heads * c.v_dim) % 64 || (c.qk_nope + c.qk_rope) % 2)
+    return MLA_OK;
+  const WeightLayout& L = h->L;
+  const char* b = h->base;
+  const int H = c.n_heads, dn = c.qk_nope, dv = c.v_dim, rkv = c.kv_lora_rank, D = c.hidden, rq = c.q_lora_rank;
+  int st = MLA_OK;
+  st |= make_map2(&T.a_W1, b + L.W1, D, L.N1, D, 128);
+  if (rq) st |= make_map2(&T.a_Wqb, b + L.Wqb, rq, L.Hq, rq, 128);
+  st |= make_map(&T.a_Wuk, b + L.Wuk, dn, rkv, H, (long long)dn * 2, (long long)rkv * dn * 2, 128, 0);
+  st |= make_map(&T.a_Wuv, b + L.Wuv, rkv, dv, H, (long long)rkv * 2, (long long)dv * rkv * 2, 128, 0);
+  st |= make_map2(&T.a_Wo, b + L.Wo, (long long)H * dv, D, (long long)H * dv, 128);
+  st |= make_map2(&T.b_W1, b + L.W1, D, L.N1, D, 256);
+  st |= make_map2(&T.b_W1q, b + L.W1, D, L.Nq1, D, 256);
+  st |= make_map2(&T.b_W1kv, b + L.W1 + (size_t)L.Nq1 * D * 2, D, L.R, D, 256);
+  if (rq) st |= make_map2(&T.b_Wqb, b + L.Wqb, rq, L.Hq, rq, 256);
+  st |= make_map2(&T.b_Wkvb, b + L.Wkvb, rkv, L.Hkv, rkv, 256);
+  st |= make_map2(&T.b_Wo, b + L.Wo, (long long)H * dv, D, (long long)H * dv, 256);
+  if (st != MLA_OK) return MLA_OK;   // stay on the CUDA-core path
+  T.enabled = 1;
+  return MLA_OK;
+}
+
+static inline bool tc_decode_qkv_supported(const mla_handle* h, int n) { return h->tc.enabled && n <= 256; }
+static inline bool tc_decode_attn_supported(const mla_handle* h, int n, int) { return h->tc.enabled && n <= 256; }
+static inline bool tc_prefill_supported(const mla_handle* h, int) { return h->tc.enabled; }
+
+static GemmArgs gemm_args(int M, int N, int K, int batches, int mode, void* out, long long ldo, long long bstride,
+                          int* flag) {
+  GemmArgs g{};
+  g.M = M; g.N = N; g.K = K; g.batches = batches; g.mode = mode; g.out = out; g.ldo = ldo; g.bstride = bstride;
+  g.flag = flag;
+  return g;
+}
+
+static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, const float* cos, const float* sin,
+                                void* kv_cache, int n_blocks, const int32_t* slot_mapping, void* q_abs, void* q_pe,
+                                char* ws, size_t tc_off, cudaStream_t s) {
+  const mla_config& c = h->cfg;
+  const WeightLayout& L = h->L;
+  const TcState& T = h->tc;
+  const TcDecodeWs W = tc_decode_ws(h, n);
+  char* tw = ws + tc_off;
+  int* flag = (int*)ws;
+  const int H = c.n_heads, dn = c.qk_nope, dr = c.qk_rope, rkv = c.kv_lora_rank, D = c.hidden, rq = c.q_lora_rank;
+  const int bn = pick_bn(n);
+  int st;
+  // 1. Yp[split] = x @ W1 (swap-AB: A = W1 [N1, D], B = x [n, D])
+  CUtensorMap mx;
+  if ((st = make_map2(&mx, hidden, D, n, D, bn)) != MLA_OK) return st;
+  GemmArgs g = gemm_args(L.N1, n, D, 1, EPI_F32_T, tw + W.Yp, L.N1, 0, flag);
+  if ((st = launch_gemm(T.a_W1, mx, g, bn, W.s1, T.num_sms, s)) != MLA_OK) return st;
+  // 2. split sum, norms, RoPE, scatter (and, without q_lora, q_nope / q_pe)
+  FrontFoldTcArgs f{};
+  f.Yp = (const float*)(tw + W.Yp); f.split_stride = (long long)n * L.N1; f.splits = W.s1; f.N1 = L.N1;
+  f.rq = rq; f.Nq1 = L.Nq1; f.rkv = rkv; f.dr = dr; f.H = H; f.dn = dn;
+  f.q_norm_w = rq ? (const float*)(h->base + L.gq) : nullptr;
+  f.kv_norm_w = (const float*)(h->base + L.gkv); f.eps = c.norm_eps;
+  f.cos = cos; f.sin = sin;
+  f.qn = (bf16*)(tw + W.qn); f.q_nope = (bf16*)(tw + W.q_nope); f.q_pe = (bf16*)q_pe;
+  f.cache = (bf16*)kv_cache; f.n_rows = (long long)n_blocks * c.block_size; f.slot = slot_mapping;
+  f.layout = c.row_layout; f.flag = flag;
+  const size_t ff_smem = (size_t)L.N1 * 4;
+  if (ff_smem > 48 * 1024) cudaFuncSetAttribute(frontfold_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ff_smem);
+  frontfold_tc_kernel<<<n, 256, ff_smem, s>>>(f);
+  mla_count_launch(1);
+  // 3. q = qn @ wq_b with q_nope out and RoPE(q_pe) out (swap-AB)
+  if (rq) {
+    CUtensorMap mq;
+    if ((st = make_map2(&mq, tw + W.qn, rq, n, rq, bn)) != MLA_OK) return st;
+    GemmArgs g2 = gemm_args(L.Hq, n, rq, 1, EPI_QROPE_T, tw + W.q_nope, 0, 0, flag);
+    g2.out2 = q_pe; g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr;
+    if ((st = launch_gemm(T.a_Wqb, mq, g2, bn, 1, T.num_sms, s)) != MLA_OK) return st;
+  }
+  // 4. q_abs[h] = q_nope[h] @ W_UK[h]  (batched over heads: A = Wuk[h] [r_kv, d_n], B = q_nope[:, h, :])
+  CUtensorMap mn;
+  if ((st = make_map(&mn, tw + W.q_nope, dn, H, n, (long long)dn * 2, (long long)H * dn * 2, bn, 1)) != MLA_OK)
+    return st;
+  GemmArgs g3 = gemm_args(rkv, n, dn, H, EPI_BF16_T, q_abs, (long long)H * rkv, rkv, flag);
+  g3.b_rows_dim2 = 1;
+  return launch_gemm(T.a_Wuk, mn, g3, bn, 1, T.num_sms, s);
+}
+
+static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const void* q_pe, const void* kv_cache,
+                                 int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
+                                 int max_ctx, int n, void* out, void* head, char* ws, size_t tc_off,
+                                 cudaStream_t s, float* part_o, float* part_ml, int splits, bf16* o_lat) {
+  const mla_config& c = h->cfg;
+  const TcState& T = h->tc;
+  const TcDecodeWs W = tc_decode_ws(h, n);
+  char* tw = ws + tc_off;
+  int* flag = (int*)ws;
+  const int H = c.n_heads, dr = c.qk_rope, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
+  const int bn = pick_bn(n);
+  int st;
+  // 1. split-KV absorbed attention (CUDA cores) and the LSE merge -> o_lat (bf16)
+  AttnArgs p{};
+  p.q_abs = q_abs; p.q_pe = q_pe; p.cache = kv_cache; p.n_blocks = n_blocks; p.bs = c.block_size;
+  p.block_table = block_table; p.mbps = mbps; p.ctx = ctx; p.max_ctx = max_ctx;
+  p.H = H; p.r_kv = rkv; p.d_r = dr; p.layout = c.row_layout; p.scale = h->scale;
+  p.n_splits = splits; p.chunk = (int)cdiv(cdiv(max_ctx, splits), ATT_TR) * ATT_TR;
+  p.part_o = part_o; p.part_ml = part_ml; p.flag = flag;
+  const int R = rkv + dr;
+  const size_t smem = (size_t)(ATT_TR * (R + 1) + ATT_HPB * R) * 4;
+  cudaFuncSetAttribute(attn_decode_simt_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  mla_timer_begin("attn", s);
+  attn_decode_simt_kernel<bf16><<<dim3(splits, n, (unsigned)cdiv(H, ATT_HPB)), 256, smem, s>>>(p);
+  mla_timer_end("attn", s);
+  mla_count_launch(1);
+  attn_combine_kernel<bf16><<<dim3(n, H), 128, 0, s>>>(part_o, part_ml, splits, H, rkv, o_lat);
+  mla_count_launch(1);
+  // 2. head_out[h] = o_lat[h] @ W_UV[h]  (A = Wuv[h] [d_v, r_kv], B = o_lat[:, h, :])
+  CUtensorMap mo;
+  if ((st = make_map(&mo, o_lat, rkv, H, n, (long long)rkv * 2, (long long)H * rkv * 2, bn, 1)) != MLA_OK) return st;
+  GemmArgs g4 = gemm_args(dv, n, rkv, H, EPI_BF16_T, head, (long long)H * dv, dv, flag);
+  g4.b_rows_dim2 = 1;
+  if ((st = launch_gemm(T.a_Wuv, mo, g4, bn, 1, T.num_sms, s)) != MLA_OK) return st;
+  // 3. out = head_out @ wo  (swap-AB, K split, then reduce to bf16)
+  CUtensorMap mh;
+  if ((st = make_map2(&mh, head, (long long)H * dv, n, (long long)H * dv, bn)) != MLA_OK) return st;
+  GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
+  if ((st = launch_gemm(T.a_Wo, mh, g5, bn, W.s5, T.num_sms, s)) != MLA_OK) return st;
+  const long long cnt = (long long)n * D;
+  splitk_reduce_bf16_kernel<<<(unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s>>>(
+      (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);
+  mla_count_launch(1);
+  return MLA_OK;
+}
+
+static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, const float* cos, const float* sin,
+                             void* out, void* head, void* kv_cache, int n_blocks, const int32_t* slot_mapping,
+                             char* ws, size_t pY1, size_t pqn, size_t pQ, size_t pcn, size_t pkpe, size_t pKV,
+                             cudaStream_t s) {
+  const mla_config& c = h->cfg;
+  const WeightLayout& L = h->L;
+  const TcState& T = h->tc;
+  int* flag = (int*)ws;
+  const int H = c.n_heads, dn = c.qk_nope, dr = c.qk_rope, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
+  const int rq = c.q_lora_rank;
+  int st;
+  CUtensorMap mx;
+  if ((st = make_map2(&mx, hidden, D, S, D, 128)) != MLA_OK) return st;
+  float* Y1 = (float*)(ws + pY1);
+  bf16* Q = (bf16*)(ws + pQ);
+  FrontFoldArgs f{};
+  if (rq) {
+    GemmArgs g = gemm_args(S, L.N1, D, 1, EPI_F32_N, Y1, L.N1, 0, flag);
+    if ((st = launch_gemm(mx, T.b_W1, g, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+    f.Y = Y1; f.ldy = L.N1; f.kv0 = L.Nq1;
+  } else {
+    GemmArgs gq = gemm_args(S, L.Hq, D, 1, EPI_QROPE_N, Q, L.Hq, 0, flag);
+    gq.cos = cos; gq.sin = sin; gq.H = H; gq.dn = dn; gq.dr = dr;
+    if ((st = launch_gemm(mx, T.b_W1q, gq, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+    GemmArgs gk = gemm_args(S, L.R, D, 1, EPI_F32_N, Y1, L.R, 0, flag);
+    if ((st = launch_gemm(mx, T.b_W1kv, gk, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+    f.Y = Y1; f.ldy = L.R; f.kv0 = 0;
+  }
+  f.r_q = rq; f.r_kv = rkv; f.d_r = dr;
+  f.q_norm_w = rq ? (const float*)(h->base + L.gq) : nullptr;
+  f.kv_norm_w = (const float*)(h->base + L.gkv); f.eps = c.norm_eps;
+  f.cos = cos; f.sin = sin;
+  f.qn = rq ? ws + pqn : nullptr; f.ldqn = rq;
+  f.cache = kv_cache; f.n_rows = (long long)n_blocks * c.block_size;
+  f.slot = slot_mapping; f.layout = c.row_layout; f.flag = flag;
+  f.cn = ws + pcn; f.kpe = ws + pkpe;
+  frontfold_epilogue_kernel<bf16><<<S, 256, 0, s>>>(f);
+  mla_count_launch(1);
+  if (rq) {
+    CUtensorMap mq;
+    if ((st = make_map2(&mq, ws + pqn, rq, S, rq, 128)) != MLA_OK) return st;
+    GemmArgs g2 = gemm_args(S, L.Hq, rq, 1, EPI_QROPE_N, Q, L.Hq, 0, flag);
+    g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr;
+    if ((st = launch_gemm(mq, T.b_Wqb, g2, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+  }
+  CUtensorMap mc;
+  if ((st = make_map2(&mc, ws + pcn, rkv, S, rkv, 128)) != MLA_OK) return st;
+  bf16* KV = (bf16*)(ws + pKV);
+  GemmArgs g3 = gemm_args(S, L.Hkv, rkv, 1, EPI_BF16_N, KV, L.Hkv, 0, flag);
+  if ((st = launch_gemm(mc, T.b_Wkvb, g3, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+  PrefillAttnArgs pa{};
+  pa.Q = Q; pa.ldq = L.Hq; pa.KV = KV; pa.ldkv = L.Hkv; pa.kpe = ws + pkpe;
+  pa.O = head; pa.ldo = (long long)H * dv; pa.S = S; pa.H = H; pa.d_n = dn; pa.d_r = dr; pa.d_v = dv;
+  pa.scale = h->scale;
+  const size_t smem = (size_t)(PA_BQ * (dn + dr) + PA_BK * (dn + dr + 1) + PA_BK * dv) * 4;
+  cudaFuncSetAttribute(prefill_attn_simt_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  mla_timer_begin("prefill_attn", s);
+  prefill_attn_simt_kernel<bf16><<<dim3((unsigned)cdiv(S, PA_BQ), H), 128, smem, s>>>(pa);
+  mla_timer_end("prefill_attn", s);
+  mla_count_launch(1);
+  CUtensorMap mh;
+  if ((st = make_map2(&mh, head, (long long)H * dv, S, (long long)H * dv, 128)) != MLA_OK) return st;
+  GemmArgs g5 = gemm_args(S, D, H * dv, 1, EPI_BF16_N, out, D, 0, flag);
+  return launch_gemm(mh, T.b_Wo, g5, 256, 1, T.num_sms, s);
+}

@@ -1,6 +1,14 @@
-// What the tensor-core (tcgen05) path keeps per layer handle.
+// What the tensor-core (tcgen05) path keeps per layer handle: TMA tensor maps
+// of the repacked weights (built once at init) and the device's SM count.
 #pragma once
 
+#include <cuda.h>
+
 struct TcState {
-  int enabled;
+  int enabled;       // bf16 activations with bf16 weights on an sm_100 device
+  int num_sms;
+  // weights as the A operand (decode, swap-AB): 128-row boxes
+  CUtensorMap a_W1, a_Wqb, a_Wuk, a_Wuv, a_Wo;
+  // weights as the B operand (prefill): 256-row boxes
+  CUtensorMap b_W1q, b_W1kv, b_W1, b_Wqb, b_Wkvb, b_Wo;
 };
