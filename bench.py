@@ -392,7 +392,13 @@ def run_ours(args, world, rank, local):
         barrier(world)
         torch.cuda.synchronize()
         clocks = ClockSampler(local)
+        t_soak = time.perf_counter()            # keep the GPU busy long enough for the
+        while time.perf_counter() - t_soak < 1.0:   # clock sampler to see it under load
+            g.replay()
+            torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("mla_timed_steps")
         times = timed_replays(g, args.steps, flush, stream)
+        torch.cuda.nvtx.range_pop()
         clk = clocks.stop()
         barrier(world)
         torch.cuda.synchronize()

@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(192, 1)
       int mt, nt, b, s;
       decode_unit(g, u, mt, nt, b, s);
       const int acc = tile & 1, use = tile >> 1;
-      if (!mbar_wait(tfull_bar(acc), use & 1, abort_word, g.flag)) break;
+      if (!mbar_wait_warp(tfull_bar(acc), use & 1, abort_word, g.flag)) break;
       tc_fence_after();
       const int m = mt * C::BM + warp * 32 + lane;
       const uint32_t row_addr = tmem + ((uint32_t)(warp * 32) << 16) + acc * BN;

@@ -9,6 +9,7 @@
 #include "handle.cuh"
 #include "simt_kernels.cuh"
 #include "tc_gemm.cuh"
+#include "tc_attn.cuh"
 
 namespace mla {
 namespace tc {
@@ -333,20 +334,56 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   const int H = c.n_heads, dr = c.qk_rope, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
   const int bn = pick_bn(n);
   int st;
-  // 1. split-KV absorbed attention (CUDA cores) and the LSE merge -> o_lat (bf16)
-  AttnArgs p{};
-  p.q_abs = q_abs; p.q_pe = q_pe; p.cache = kv_cache; p.n_blocks = n_blocks; p.bs = c.block_size;
-  p.block_table = block_table; p.mbps = mbps; p.ctx = ctx; p.max_ctx = max_ctx;
-  p.H = H; p.r_kv = rkv; p.d_r = dr; p.layout = c.row_layout; p.scale = h->scale;
-  p.n_splits = splits; p.chunk = (int)cdiv(cdiv(max_ctx, splits), ATT_TR) * ATT_TR;
-  p.part_o = part_o; p.part_ml = part_ml; p.flag = flag;
+  // 1. split-KV absorbed attention and the LSE merge -> o_lat (bf16)
   const int R = rkv + dr;
-  const size_t smem = (size_t)(ATT_TR * (R + 1) + ATT_HPB * R) * 4;
-  cudaFuncSetAttribute(attn_decode_simt_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  mla_timer_begin("attn", s);
-  attn_decode_simt_kernel<bf16><<<dim3(splits, n, (unsigned)cdiv(H, ATT_HPB)), 256, smem, s>>>(p);
-  mla_timer_end("attn", s);
-  mla_count_launch(1);
+  const bool tc_attn = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && H <= 128;
+  if (tc_attn) {
+    // (sequence, split) clusters: about three waves of CTA pairs, at most the
+    // splits the workspace holds
+    const int pairs = T.num_sms / 2 > 0 ? T.num_sms / 2 : 74;
+    int sp = (int)cdiv(3 * pairs, n);
+    if (sp > splits) sp = splits;
+    if (sp < 1) sp = 1;
+    const int chunk = (int)cdiv(cdiv(max_ctx, sp), 64) * 64;
+    sp = (int)cdiv(max_ctx, chunk);
+    splits = sp;
+    CUtensorMap mqa, mqp, mc;
+    if ((st = make_map2(&mqa, q_abs, rkv, (long long)n * H, rkv, 128)) != MLA_OK) return st;
+    if ((st = make_map2(&mqp, q_pe, dr, (long long)n * H, dr, 128)) != MLA_OK) return st;
+    if ((st = make_map2(&mc, kv_cache, R, (long long)n_blocks * c.block_size, R, 64)) != MLA_OK) return st;
+    TcAttnArgs ta{};
+    ta.n = n; ta.H = H; ta.splits = sp; ta.chunk = chunk;
+    ta.bs = c.block_size; ta.n_blocks = n_blocks; ta.mbps = mbps; ta.max_ctx = max_ctx;
+    ta.block_table = block_table; ta.ctx = ctx;
+    ta.lat_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? 0 : dr;
+    ta.rope_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? rkv : 0;
+    ta.scale_log2 = h->scale * 1.4426950408889634f;
+    ta.part_o = part_o; ta.part_ml = part_ml; ta.flag = flag;
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr[dev]) {
+      cudaFuncSetAttribute(tc_attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::SIZE);
+      attr[dev] = true;
+    }
+    mla_timer_begin("attn", s);
+    tc_attn_decode_kernel<<<2 * n * sp, 192, AttnSmem::SIZE, s>>>(mqa, mqp, mc, ta);
+    mla_timer_end("attn", s);
+    mla_count_launch(1);
+  } else {
+    AttnArgs p{};
+    p.q_abs = q_abs; p.q_pe = q_pe; p.cache = kv_cache; p.n_blocks = n_blocks; p.bs = c.block_size;
+    p.block_table = block_table; p.mbps = mbps; p.ctx = ctx; p.max_ctx = max_ctx;
+    p.H = H; p.r_kv = rkv; p.d_r = dr; p.layout = c.row_layout; p.scale = h->scale;
+    p.n_splits = splits; p.chunk = (int)cdiv(cdiv(max_ctx, splits), ATT_TR) * ATT_TR;
+    p.part_o = part_o; p.part_ml = part_ml; p.flag = flag;
+    const size_t smem = (size_t)(ATT_TR * (R + 1) + ATT_HPB * R) * 4;
+    cudaFuncSetAttribute(attn_decode_simt_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    mla_timer_begin("attn", s);
+    attn_decode_simt_kernel<bf16><<<dim3(splits, n, (unsigned)cdiv(H, ATT_HPB)), 256, smem, s>>>(p);
+    mla_timer_end("attn", s);
+    mla_count_launch(1);
+  }
   attn_combine_kernel<bf16><<<dim3(n, H), 128, 0, s>>>(part_o, part_ml, splits, H, rkv, o_lat);
   mla_count_launch(1);
   // 2. head_out[h] = o_lat[h] @ W_UV[h]  (A = Wuv[h] [d_v, r_kv], B = o_lat[:, h, :])
