@@ -3,18 +3,23 @@
 // of 64 rows.
 //
 // One 2-CTA cluster per (sequence, KV split). All heads of the token form the
-// MMA's M = 128 rows (fewer heads are padded). CTA r owns latent columns
-// [256 r, 256 r + 256); CTA 0 also owns the 64 rotary columns. Per 64-row
-// cache tile:
-//   S_r = [q_abs | q_pe]_r . tile_r^T        (tcgen05, M 128 x N 64, K 256/320)
-//   S   = S_0 + S_1                          (partials swapped through DSMEM)
-//   online softmax per head (one thread per head, nothing to reduce across
-//   threads), lazy rescale of the TMEM accumulator when the max grows by > 2^8
-//   O_r += P . V_r                           (tcgen05, M 128 x N 256, K 64,
-//                                             V = the same smem tile read MN-major)
-// so every cache byte is read from HBM once and O (128 x 512 fp32) is split
-// over the two CTAs' TMEM. Partials (unnormalised O, running max, sum) go to
-// the workspace and attn_combine_kernel merges the splits.
+// MMA's M = 128 rows (fewer heads are padded with zeros). CTA r owns latent
+// columns [256 r, 256 r + 256); CTA 0 also owns the 64 rotary columns. Per
+// 64-row cache tile:
+//   S_r = [q_abs | q_pe]_r . tile_r^T      (tcgen05, M 128 x N 64, K 256 / 320;
+//                                          the latent part of Q lives in TMEM)
+//   S   = S_0 + S_1                        (the partials swap through DSMEM)
+//   online softmax, one thread per head (nothing to reduce across threads),
+//   lazy rescale of the TMEM accumulator when the max grows by more than 2^8;
+//   P (bf16) is written back into TMEM over S
+//   O_r += P . V_r                         (tcgen05 with A = P in TMEM, M 128 x
+//                                          N 256, K 64; V = the same shared-memory
+//                                          tile read MN-major)
+// Every cache byte is read from HBM once, O (128 x 512 fp32) is split over the
+// two CTAs' TMEM, and a 4-deep ring of tiles keeps loads in flight while the
+// MMA thread issues S of later tiles ahead of P.V of earlier ones. Partials
+// (unnormalised O, reference max, sum) go to the workspace and
+// attn_combine_kernel merges the splits.
 #pragma once
 
 #include "tc_common.cuh"
@@ -27,21 +32,31 @@ struct TcAttnArgs {
   int bs, n_blocks, mbps, max_ctx;
   const int* block_table;
   const int* ctx;
+  const bf16* q_abs;   // [n, H, 512]
   int lat_col0, rope_col0;
   float scale_log2;
   float* part_o;   // [n, splits, H, 512]
   float* part_ml;  // [n, splits, H, 2]
   int* flag;
+  // optional tracing: %globaltimer stamps of cluster 0, CTA 0, for its first 64
+  // tiles, [tile][16]: softmax (head 0) 0 iteration start, 2 peer partial
+  // arrived, 3 scores summed, 4 P computed, 5 P handed over, 1 next partial sent;
+  // 8 S issued, 9 P.V issued (MMA thread); 10 tile load issued (producer);
+  // [0][15] unit start. NULL = off.
+  unsigned long long* trace;
 };
 
+constexpr int ATT_NST = 3;                      // tile ring depth
 struct AttnSmem {
-  static constexpr int Q_OFF = 0;                        // 5 x [128 x 64] bf16
-  static constexpr int TILE_OFF = 5 * 16384;             // 2 stages x 5 x [64 x 64] bf16
-  static constexpr int P_OFF = TILE_OFF + 2 * 5 * 8192;  // [128 x 64] bf16
-  static constexpr int X_OFF = P_OFF + 16384;            // [128 x 64] fp32 (peer's partial S)
-  static constexpr int BAR_OFF = X_OFF + 32768;
+  static constexpr int STAGE = 5 * 8192;        // 4 latent + 1 rope slot of [64 rows x 64 cols] bf16
+  static constexpr int TILE_OFF = 0;
+  static constexpr int QR_OFF = ATT_NST * STAGE;  // q_pe [128 x 64] bf16 (CTA 0)
+  static constexpr int X_OFF = QR_OFF + 16384;    // 2 x [128 x 64] fp32, the peer's partial S
+  static constexpr int BAR_OFF = X_OFF + 2 * 32768;
   static constexpr int SIZE = 1024 + BAR_OFF + 256;
 };
+// TMEM columns: Q latent [0,128) (bf16 pairs), S/P buffers [128,192) [192,256), O [256,512)
+constexpr uint32_t ATT_TM_Q = 0, ATT_TM_S = 128, ATT_TM_O = 256;
 
 __device__ __forceinline__ int attn_tile_rows(const TcAttnArgs& a, int b, int j0, int r1, long long* row) {
   const int blk = a.block_table[(long long)b * a.mbps + j0 / a.bs];
@@ -54,18 +69,24 @@ __device__ __forceinline__ int attn_tile_rows(const TcAttnArgs& a, int b, int j0
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_qabs, const __grid_constant__ CUtensorMap tm_qpe,
-                          const __grid_constant__ CUtensorMap tm_cache, TcAttnArgs a) {
+    tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_qpe, const __grid_constant__ CUtensorMap tm_cache,
+                          TcAttnArgs a) {
   using SM = AttnSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t q_s = sbase + SM::Q_OFF, tile_s = sbase + SM::TILE_OFF, p_s = sbase + SM::P_OFF;
-  const uint32_t x_s = sbase + SM::X_OFF, bar = sbase + SM::BAR_OFF;
-  const uint32_t full_b = bar, empty_b = bar + 16, q_full = bar + 32, s_full_b = bar + 40, s_empty_b = bar + 56;
-  const uint32_t p_full = bar + 72, o_done = bar + 80, x_full = bar + 88, x_free = bar + 96, fin = bar + 104;
-  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 128);
-  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 132);
+  const uint32_t tile_s = sbase + SM::TILE_OFF, qr_s = sbase + SM::QR_OFF, x_s = sbase + SM::X_OFF;
+  const uint32_t bar = sbase + SM::BAR_OFF;
+  // barriers (8 B each)
+  const uint32_t full_b = bar;                 // [ATT_NST] tile landed
+  const uint32_t empty_b = bar + 8 * ATT_NST;  // [ATT_NST] tile consumed by P.V
+  const uint32_t s_full_b = bar + 16 * ATT_NST;        // [2]
+  const uint32_t p_full_b = s_full_b + 16;             // [2]
+  const uint32_t sp_empty_b = p_full_b + 16;           // [2] S/P buffer free (P.V done)
+  const uint32_t q_ready = sp_empty_b + 16, qr_full = q_ready + 8, o_done = qr_full + 8;
+  const uint32_t x_full_b = o_done + 8, x_free_b = x_full_b + 16, fin = x_free_b + 16;   // x_*: [2]
+  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 192);
+  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 196);
 
   const uint32_t r = cluster_ctarank(), peer = r ^ 1u;
   const int cid = blockIdx.x >> 1;
@@ -87,19 +108,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     return;
   }
   const int nkb = (r == 0) ? 5 : 4;
+  unsigned long long* trace = (a.trace && cid == 0 && r == 0) ? a.trace : nullptr;
+  if (trace && threadIdx.x == 0) trace[15] = global_timer_ns();
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < ATT_NST; ++i) { mbar_init(full_b + 8 * i, 1); mbar_init(empty_b + 8 * i, 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(full_b + 8 * i, 1);
-      mbar_init(empty_b + 8 * i, 1);
       mbar_init(s_full_b + 8 * i, 1);
-      mbar_init(s_empty_b + 8 * i, 128);
+      mbar_init(p_full_b + 8 * i, 128);
+      mbar_init(sp_empty_b + 8 * i, 1);
     }
-    mbar_init(q_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(q_ready, 128);
+    mbar_init(qr_full, 1);
     mbar_init(o_done, 1);
-    mbar_init(x_full, 128);
-    mbar_init(x_free, 128);
+    for (int i = 0; i < 2; ++i) { mbar_init(x_full_b + 8 * i, 1); mbar_init(x_free_b + 8 * i, 4); }
     mbar_init(fin, 1);
     *abort_word = 0;
     fence_mbar_init();
@@ -110,71 +132,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   cluster_sync_all();   // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_S = tmem, tmem_O = tmem + 256;
 
   if (warp == 4) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       prefetch_tmap(&tm_cache);
-      mbar_arrive_expect_tx(q_full, nkb * 16384);
-      for (int j = 0; j < 4; ++j)
-        tma_load_3d(q_s + j * 16384, &tm_qabs, q_full, (int)r * 256 + 64 * j, b * a.H, 0);
-      if (r == 0) tma_load_3d(q_s + 4 * 16384, &tm_qpe, q_full, 0, b * a.H, 0);
+      if (r == 0) {
+        mbar_arrive_expect_tx(qr_full, 16384);
+        tma_load_3d(qr_s, &tm_qpe, qr_full, 0, b * a.H, 0);
+      }
       int t = 0;
       for (; t < T; ++t) {
-        const int st = t & 1;
-        if (!mbar_wait(empty_b + 8 * st, ((t >> 1) & 1) ^ 1, abort_word, a.flag)) break;
+        const int st = t % ATT_NST;
+        if (!mbar_wait(empty_b + 8 * st, ((t / ATT_NST) & 1) ^ 1, abort_word, a.flag)) break;
         long long row;
         if (attn_tile_rows(a, b, r0 + 64 * t, r1, &row) < 0 && r == 0) set_flag(a.flag, MLA_FLAG_BAD_BLOCK);
         mbar_arrive_expect_tx(full_b + 8 * st, nkb * 8192);
-        const uint32_t dst = tile_s + st * 5 * 8192;
+        const uint32_t dst = tile_s + st * SM::STAGE;
         for (int j = 0; j < 4; ++j)
           tma_load_3d(dst + j * 8192, &tm_cache, full_b + 8 * st, a.lat_col0 + (int)r * 256 + 64 * j, (int)row, 0);
         if (r == 0) tma_load_3d(dst + 4 * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
+        if (trace && t < 64) trace[t * 16 + 10] = global_timer_ns();
       }
       // drain the loads still in flight
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(q_full, 0)) if (global_timer_ns() - t0 > WAIT_LIMIT_NS) break;
-      for (int u = (t > 2 ? t - 2 : 0); u < t; ++u) {
+      if (r == 0) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(qr_full, 0)) if (global_timer_ns() - t0 > WAIT_LIMIT_NS) break;
+      }
+      for (int u = (t > ATT_NST ? t - ATT_NST : 0); u < t; ++u) {
         const uint64_t t1 = global_timer_ns();
-        while (!mbar_try_wait(full_b + 8 * (u & 1), (u >> 1) & 1))
+        while (!mbar_try_wait(full_b + 8 * (u % ATT_NST), (u / ATT_NST) & 1))
           if (global_timer_ns() - t1 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
       }
     }
   } else if (warp == 5) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer: S runs up to two tiles ahead of P.V ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64);
       constexpr uint32_t idesc_o = idesc_bf16(128, 256, 1);
-      bool ok = mbar_wait(q_full, 0, abort_word, a.flag);
-      auto issue_o = [&](int u) -> bool {
-        if (!mbar_wait(p_full, u & 1, abort_word, a.flag)) return false;
-        tc_fence_after();
-        const uint32_t v = tile_s + (u & 1) * 5 * 8192;
+      bool ok = mbar_wait(q_ready, 0, abort_word, a.flag);
+      if (ok && r == 0) ok = mbar_wait(qr_full, 0, abort_word, a.flag);
+      tc_fence_after();
+      int next_s = 0, next_o = 0;
+      uint64_t t_last = global_timer_ns();
+      while (ok && next_o < T) {
+        bool did = false;
+        if (next_s < T && next_s < next_o + 2) {
+          const int t = next_s, st = t % ATT_NST, sb = t & 1;
+          if (mbar_test(full_b + 8 * st, (t / ATT_NST) & 1) && mbar_test(sp_empty_b + 8 * sb, ((t >> 1) & 1) ^ 1)) {
+            tc_fence_after();
+            const uint32_t tl = tile_s + st * SM::STAGE;
+            const uint32_t d = tmem + ATT_TM_S + 64 * sb;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(tmem_O, sdesc_sw128(p_s + 32 * k), sdesc_sw128_mn(v + 2048 * k, 8192), idesc_o,
-                   (u > 0 || k > 0) ? 1u : 0u);
-        mma_commit(o_done);
-        mma_commit(empty_b + 8 * (u & 1));
-        return true;
-      };
-      int t = 0;
-      for (; ok && t < T; ++t) {
-        const int sb = t & 1;
-        if (!mbar_wait(s_empty_b + 8 * sb, ((t >> 1) & 1) ^ 1, abort_word, a.flag)) { ok = false; break; }
-        if (!mbar_wait(full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tl = tile_s + sb * 5 * 8192;
-        for (int j = 0; j < nkb; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tmem_S + sb * 64, sdesc_sw128(q_s + j * 16384 + 32 * k), sdesc_sw128(tl + j * 8192 + 32 * k),
-                     idesc_s, (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(s_full_b + 8 * sb);
-        if (t >= 1 && !issue_o(t - 1)) { ok = false; break; }
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ts(d, tmem + ATT_TM_Q + 32 * j + 8 * k, sdesc_sw128(tl + j * 8192 + 32 * k), idesc_s,
+                            (j > 0 || k > 0) ? 1u : 0u);
+            if (r == 0) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_bf16(d, sdesc_sw128(qr_s + 32 * k), sdesc_sw128(tl + 4 * 8192 + 32 * k), idesc_s, 1u);
+            }
+            mma_commit(s_full_b + 8 * sb);
+            if (trace && t < 64) trace[t * 16 + 8] = global_timer_ns();
+            ++next_s;
+            did = true;
+          }
+        }
+        if (!did && next_o < next_s) {
+          const int u = next_o, st = u % ATT_NST, sb = u & 1;
+          if (mbar_test(p_full_b + 8 * sb, (u >> 1) & 1)) {
+            tc_fence_after();
+            const uint32_t v = tile_s + st * SM::STAGE;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ts(tmem + ATT_TM_O, tmem + ATT_TM_S + 64 * sb + 8 * k, sdesc_sw128_mn(v + 2048 * k, 8192),
+                          idesc_o, (u > 0 || k > 0) ? 1u : 0u);
+            mma_commit(o_done);
+            mma_commit(sp_empty_b + 8 * sb);
+            mma_commit(empty_b + 8 * st);
+            if (trace && u < 64) trace[u * 16 + 9] = global_timer_ns();
+            ++next_o;
+            did = true;
+          }
+        }
+        if (did) {
+          t_last = global_timer_ns();
+        } else if (*abort_word) {
+          ok = false;
+        } else if (global_timer_ns() - t_last > WAIT_LIMIT_NS) {
+          *abort_word = 1;
+          set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT);
+          ok = false;
+        }
       }
-      if (ok) issue_o(T - 1);
       mma_commit(fin);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(fin, 0))
@@ -184,101 +236,131 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     // ---------------- softmax: thread h <-> head h <-> TMEM lane h ----------------
     const int h = threadIdx.x;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // Q latent half of head h -> TMEM (bf16 pairs), zero for padding heads
+    {
+      const uint4* src = (const uint4*)(a.q_abs + ((long long)b * a.H + (h < a.H ? h : 0)) * 512 + r * 256);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t q[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 v = (h < a.H) ? src[4 * c + k] : make_uint4(0, 0, 0, 0);
+          q[4 * k] = v.x; q[4 * k + 1] = v.y; q[4 * k + 2] = v.z; q[4 * k + 3] = v.w;
+        }
+        tmem_st16(tmem + ATT_TM_Q + lane_base + 16 * c, q);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(q_ready);
+    }
+    // partial-score exchange: S_r(k) goes with st.async into the peer's X[k & 1],
+    // completing bytes on the peer's x_full[k & 1]; each peer warp frees the
+    // buffer with one remote arrive on our x_free[k & 1] once it has read it.
     const uint32_t peer_x = mapa_shared(x_s + h * 256, peer);
-    const uint32_t peer_x_full = mapa_shared(x_full, peer), peer_x_free = mapa_shared(x_free, peer);
-    const float4* xloc = (const float4*)(smem + SM::X_OFF + h * 256);
-    uint8_t* prow = smem + SM::P_OFF + h * 128;
+    const uint32_t peer_x_full = mapa_shared(x_full_b, peer), peer_x_free = mapa_shared(x_free_b, peer);
+    float v[64];   // own partial of the tile processed next (already sent to the peer)
+    auto load_and_send = [&](int k) -> bool {
+      const int kb = k & 1;
+      if (!mbar_wait_warp(s_full_b + 8 * kb, (k >> 1) & 1, abort_word, a.flag)) return false;
+      tc_fence_after();
+      const uint32_t sa = tmem + ATT_TM_S + 64 * kb + lane_base;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld16(sa + 16 * c, (uint32_t*)&v[16 * c]);
+      tmem_ld_wait();
+      if (!mbar_wait_cluster_warp(x_free_b + 8 * kb, ((k >> 1) & 1) ^ 1, abort_word, a.flag)) return false;
+      const uint32_t dst = peer_x + kb * 32768, bar_k = peer_x_full + 8 * kb;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)   // chunk c of row h at slot c ^ (h & 15): no bank conflicts
+        st_async_v4(dst + 16 * (c ^ (h & 15)), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], bar_k);
+      return true;
+    };
     float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
+    bool ok = load_and_send(0);
     for (int t = 0; t < T && ok; ++t) {
-      const int sb = t & 1;
+      const int sb = t & 1, st = t % ATT_NST;
       long long row_unused;
       int valid = attn_tile_rows(a, b, r0 + 64 * t, r1, &row_unused);
       if (valid < 0) valid = 0;
-      if (!mbar_wait_warp(s_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      tc_fence_after();
-      float s[64];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(tmem_S + sb * 64 + lane_base + 16 * c, (uint32_t*)&s[16 * c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(s_empty_b + 8 * sb);
-      // swap partial scores with the peer CTA
-      if (t >= 1 && !mbar_wait_cluster_warp(x_free, (t - 1) & 1, abort_word, a.flag)) { ok = false; break; }
-#pragma unroll
-      for (int c = 0; c < 16; ++c)   // chunk c of row h lives at slot c ^ (h & 15): no bank conflicts
-        st_cluster_v4(peer_x + 16 * (c ^ (h & 15)), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
-      mbar_arrive_remote(peer_x_full);
-      if (!mbar_wait_cluster_warp(x_full, t & 1, abort_word, a.flag)) { ok = false; break; }
+      const bool tr = trace && h == 0 && t < 64;
+      if (tr) trace[t * 16 + 0] = global_timer_ns();
+      if (h == 0) mbar_arrive_expect_tx(x_full_b + 8 * sb, 32768);
+      if (!mbar_wait_warp(x_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (tr) trace[t * 16 + 2] = global_timer_ns();
+      const float4* xloc = (const float4*)(smem + SM::X_OFF + sb * 32768 + h * 256);
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float4 v = xloc[c ^ (h & 15)];
-        s[4 * c] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
+        const float4 x = xloc[c ^ (h & 15)];
+        v[4 * c] += x.x; v[4 * c + 1] += x.y; v[4 * c + 2] += x.z; v[4 * c + 3] += x.w;
       }
-      mbar_arrive_remote(peer_x_free);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(peer_x_free + 8 * sb);
+      if (tr) trace[t * 16 + 3] = global_timer_ns();
       // online softmax in log2 units with a lazily moved reference max
-      float mt = -INFINITY;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        s[j] = (j < valid) ? s[j] * a.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[j]);
-      }
+      for (int j = 0; j < 64; ++j)
+        if (j < valid) m4[j & 3] = fmaxf(m4[j & 3], v[j]);
+      const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
       if (mt > m_ref + 8.f) {
-        if (m_ref != -INFINITY) { alpha = exp2f(m_ref - mt); rescale = true; }
+        if (m_ref != -INFINITY) { alpha = ex2_approx(m_ref - mt); rescale = true; }
         m_ref = mt;
       }
-      float psum = 0.f;
+      const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
-        const float p0 = (m_ref == -INFINITY) ? 0.f : exp2f(s[j] - m_ref);
-        const float p1 = (m_ref == -INFINITY) ? 0.f : exp2f(s[j + 1] - m_ref);
+        const float p0 = (j < valid) ? ex2_approx(fmaf(v[j], a.scale_log2, nm)) : 0.f;
+        const float p1 = (j + 1 < valid) ? ex2_approx(fmaf(v[j + 1], a.scale_log2, nm)) : 0.f;
         __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        psum += __low2float(pb) + __high2float(pb);
+        ps[(j >> 1) & 3] += __low2float(pb) + __high2float(pb);
         pk[j >> 1] = *reinterpret_cast<uint32_t*>(&pb);
       }
-      // O(t-1) complete: P may be overwritten and O rescaled
-      if (t >= 1 && !mbar_wait_warp(o_done, (t - 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      tc_fence_after();
+      const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      if (tr) trace[t * 16 + 4] = global_timer_ns();
       if (__any_sync(0xffffffffu, rescale) && t >= 1) {
+        // P.V of the previous tiles must be complete before O is touched
+        if (!mbar_wait_warp(o_done, (t - 1) & 1, abort_word, a.flag)) { ok = false; break; }
+        tc_fence_after();
         for (int c = 0; c < 16; ++c) {
           uint32_t o[16];
-          tmem_ld16(tmem_O + lane_base + 16 * c, o);
+          tmem_ld16(tmem + ATT_TM_O + lane_base + 16 * c, o);
           tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st16(tmem_O + lane_base + 16 * c, o);
+          tmem_st16(tmem + ATT_TM_O + lane_base + 16 * c, o);
         }
-        tmem_st_wait();
       }
       l = l * alpha + psum;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = v;
-      }
       if (valid < 64) {
         // rows past the context may hold anything (even NaN); P is 0 there, but
         // 0 * NaN is not, so clear them in the four latent slots before P.V
-        uint8_t* tl = smem + SM::TILE_OFF + (t & 1) * 5 * 8192;
+        uint8_t* tl = smem + SM::TILE_OFF + st * SM::STAGE;
         const int nbytes = (64 - valid) * 128;
         for (int i = h * 16; i < 4 * nbytes; i += 128 * 16) {
           const int j = i / nbytes, off = i % nbytes;
           *reinterpret_cast<uint4*>(tl + j * 8192 + valid * 128 + off) = make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
+      const uint32_t sp_addr = tmem + ATT_TM_S + 64 * sb + lane_base;
+      tmem_st16(sp_addr, pk);            // P over S: 32 columns of bf16 pairs
+      tmem_st16(sp_addr + 16, pk + 16);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full_b + 8 * sb);
+      if (tr) trace[t * 16 + 5] = global_timer_ns();
+      if (t + 1 < T && !load_and_send(t + 1)) { ok = false; break; }
+      if (tr) trace[t * 16 + 1] = global_timer_ns();
     }
     if (ok && mbar_wait_warp(o_done, (T - 1) & 1, abort_word, a.flag)) {
       tc_fence_after();
       float* po = a.part_o + (unit * a.H + h) * 512 + r * 256;
       for (int c = 0; c < 16; ++c) {
         uint32_t o[16];
-        tmem_ld16(tmem_O + lane_base + 16 * c, o);
+        tmem_ld16(tmem + ATT_TM_O + lane_base + 16 * c, o);
         tmem_ld_wait();
         if (h < a.H) {
 #pragma unroll

@@ -336,7 +336,8 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   int st;
   // 1. split-KV absorbed attention and the LSE merge -> o_lat (bf16)
   const int R = rkv + dr;
-  const bool tc_attn = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && H <= 128;
+  const bool tc_attn = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && H <= 128 &&
+                       (((uintptr_t)q_abs) & 15) == 0;
   if (tc_attn) {
     // (sequence, split) clusters: about three waves of CTA pairs, at most the
     // splits the workspace holds
@@ -347,14 +348,13 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
     const int chunk = (int)cdiv(cdiv(max_ctx, sp), 64) * 64;
     sp = (int)cdiv(max_ctx, chunk);
     splits = sp;
-    CUtensorMap mqa, mqp, mc;
-    if ((st = make_map2(&mqa, q_abs, rkv, (long long)n * H, rkv, 128)) != MLA_OK) return st;
+    CUtensorMap mqp, mc;
     if ((st = make_map2(&mqp, q_pe, dr, (long long)n * H, dr, 128)) != MLA_OK) return st;
     if ((st = make_map2(&mc, kv_cache, R, (long long)n_blocks * c.block_size, R, 64)) != MLA_OK) return st;
     TcAttnArgs ta{};
     ta.n = n; ta.H = H; ta.splits = sp; ta.chunk = chunk;
     ta.bs = c.block_size; ta.n_blocks = n_blocks; ta.mbps = mbps; ta.max_ctx = max_ctx;
-    ta.block_table = block_table; ta.ctx = ctx;
+    ta.block_table = block_table; ta.ctx = ctx; ta.q_abs = (const bf16*)q_abs;
     ta.lat_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? 0 : dr;
     ta.rope_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? rkv : 0;
     ta.scale_log2 = h->scale * 1.4426950408889634f;
@@ -367,7 +367,7 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
       attr[dev] = true;
     }
     mla_timer_begin("attn", s);
-    tc_attn_decode_kernel<<<2 * n * sp, 192, AttnSmem::SIZE, s>>>(mqa, mqp, mc, ta);
+    tc_attn_decode_kernel<<<2 * n * sp, 192, AttnSmem::SIZE, s>>>(mqp, mc, ta);
     mla_timer_end("attn", s);
     mla_count_launch(1);
   } else {
