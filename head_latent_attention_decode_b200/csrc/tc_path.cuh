@@ -10,6 +10,7 @@
 #include "simt_kernels.cuh"
 #include "tc_gemm.cuh"
 #include "tc_attn.cuh"
+#include "tc_prefill_attn.cuh"
 
 namespace mla {
 namespace tc {
@@ -454,16 +455,38 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
   bf16* KV = (bf16*)(ws + pKV);
   GemmArgs g3 = gemm_args(S, L.Hkv, rkv, 1, EPI_BF16_N, KV, L.Hkv, 0, flag);
   if ((st = launch_gemm(mc, T.b_Wkvb, g3, 256, 1, T.num_sms, s)) != MLA_OK) return st;
-  PrefillAttnArgs pa{};
-  pa.Q = Q; pa.ldq = L.Hq; pa.KV = KV; pa.ldkv = L.Hkv; pa.kpe = ws + pkpe;
-  pa.O = head; pa.ldo = (long long)H * dv; pa.S = S; pa.H = H; pa.d_n = dn; pa.d_r = dr; pa.d_v = dv;
-  pa.scale = h->scale;
-  const size_t smem = (size_t)(PA_BQ * (dn + dr) + PA_BK * (dn + dr + 1) + PA_BK * dv) * 4;
-  cudaFuncSetAttribute(prefill_attn_simt_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  mla_timer_begin("prefill_attn", s);
-  prefill_attn_simt_kernel<bf16><<<dim3((unsigned)cdiv(S, PA_BQ), H), 128, smem, s>>>(pa);
-  mla_timer_end("prefill_attn", s);
-  mla_count_launch(1);
+  if (dn == 128 && dr == 64 && dv == 128) {
+    CUtensorMap mq, mkv, mkpe;
+    if ((st = make_map2(&mq, Q, L.Hq, S, L.Hq, 128)) != MLA_OK) return st;
+    if ((st = make_map2(&mkv, KV, L.Hkv, S, L.Hkv, 128)) != MLA_OK) return st;
+    if ((st = make_map2(&mkpe, ws + pkpe, dr, S, dr, 128)) != MLA_OK) return st;
+    TcPrefillAttnArgs pa{};
+    pa.S = S; pa.H = H; pa.q_tiles = (int)cdiv(S, 128);
+    pa.scale_log2 = h->scale * 1.4426950408889634f;
+    pa.out = (bf16*)head; pa.flag = flag;
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr[dev]) {
+      cudaFuncSetAttribute(tc_prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PaSmem::SIZE);
+      attr[dev] = true;
+    }
+    mla_timer_begin("prefill_attn", s);
+    tc_prefill_attn_kernel<<<pa.q_tiles * H, 192, PaSmem::SIZE, s>>>(mq, mkv, mkpe, pa);
+    mla_timer_end("prefill_attn", s);
+    mla_count_launch(1);
+  } else {
+    PrefillAttnArgs pa{};
+    pa.Q = Q; pa.ldq = L.Hq; pa.KV = KV; pa.ldkv = L.Hkv; pa.kpe = ws + pkpe;
+    pa.O = head; pa.ldo = (long long)H * dv; pa.S = S; pa.H = H; pa.d_n = dn; pa.d_r = dr; pa.d_v = dv;
+    pa.scale = h->scale;
+    const size_t smem = (size_t)(PA_BQ * (dn + dr) + PA_BK * (dn + dr + 1) + PA_BK * dv) * 4;
+    cudaFuncSetAttribute(prefill_attn_simt_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    mla_timer_begin("prefill_attn", s);
+    prefill_attn_simt_kernel<bf16><<<dim3((unsigned)cdiv(S, PA_BQ), H), 128, smem, s>>>(pa);
+    mla_timer_end("prefill_attn", s);
+    mla_count_launch(1);
+  }
   CUtensorMap mh;
   if ((st = make_map2(&mh, head, (long long)H * dv, S, (long long)H * dv, 128)) != MLA_OK) return st;
   GemmArgs g5 = gemm_args(S, D, H * dv, 1, EPI_BF16_N, out, D, 0, flag);
