@@ -35,8 +35,10 @@ SYMBOLS = (
     "mla_weights_bytes", "mla_init_weights", "mla_destroy", "mla_workspace_bytes",
     "mla_workspace_init", "mla_read_device_flag", "mla_clear_device_flag", "mla_rope_cos_sin",
     "mla_decode_qkv", "mla_decode_attn", "mla_prefill", "mla_strerror",
-    "mla_kernel_launch_count", "mla_set_kernel_timer",
+    "mla_kernel_launch_count", "mla_set_kernel_timer", "mla_decode_qkv_noalloc",
 )
+
+MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class mla_config(ctypes.Structure):
@@ -98,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.mla_kernel_launch_count.restype = ctypes.c_uint64
         L.mla_kernel_launch_count.argtypes = []
         L.mla_set_kernel_timer.restype = i
+        L.mla_decode_qkv_noalloc.restype = i
+        L.mla_decode_qkv_noalloc.argtypes = [vp, vp, i, vp, vp, vp, i, vp, vp, vp, vp]
         L.mla_set_kernel_timer.argtypes = [ctypes.c_char_p, vp, vp]
         _lib = L
     return _lib
@@ -192,6 +196,16 @@ def mla_decode_qkv(handle, hidden, cos, sin, kv_cache, slot_mapping, q_abs, q_pe
                                 kv_cache.shape[0], _ptr(slot_mapping), _ptr(q_abs), _ptr(q_pe),
                                 _ptr(input_norm_w), _ptr(ws), _nbytes(ws), _stream(stream)),
            "mla_decode_qkv")
+
+
+def mla_decode_qkv_noalloc(handle, hidden, cos, sin, kv_cache, slot_mapping, q_abs, q_pe,
+                           stream=None) -> None:
+    """mla_decode_qkv with the library's own fixed device scratch instead of a
+    caller workspace (for callers that cannot allocate)."""
+    n = hidden.shape[0]
+    _check(lib().mla_decode_qkv_noalloc(handle, _ptr(hidden), n, _ptr(cos), _ptr(sin), _ptr(kv_cache),
+                                        kv_cache.shape[0], _ptr(slot_mapping), _ptr(q_abs), _ptr(q_pe),
+                                        _stream(stream)), "mla_decode_qkv_noalloc")
 
 
 def mla_decode_attn(handle, q_abs, q_pe, kv_cache, block_table, context_lens, max_context_len,

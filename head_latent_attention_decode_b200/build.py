@@ -16,7 +16,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libmla_b200.so")
-SOURCES = [os.path.join(PKG, "csrc", "mla_abi.cu")]
+SOURCES = [os.path.join(PKG, "csrc", "mla_abi.cu"), os.path.join(PKG, "csrc", "mla_noalloc.cu")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

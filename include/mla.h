@@ -210,6 +210,29 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe,
                     int max_context_len, int n, void* out, void* head_out, void* ws,
                     size_t ws_bytes, void* stream);
 
+/* Size of the device array mla_decode_qkv_noalloc() uses as its workspace. */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* mla_decode_qkv without a workspace argument and without allocating: for
+ * callers that cannot allocate device memory -- a process whose device memory
+ * is entirely reserved up front by its own pool allocator, or a serving loop
+ * that must not call cudaMalloc because it synchronises the device and stalls
+ * every stream. (The pages have no counterpart; this is a library convenience.)
+ * Same computation, arguments and results as mla_decode_qkv (input_norm_w is
+ * taken as NULL); the scratch is a static device array of
+ * MLA_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
+ * process exits. The first call on a device looks up that array's address
+ * (cudaGetSymbolAddress) with the device current; make that first call before
+ * any stream capture. Returns MLA_ERR_WORKSPACE when
+ * mla_workspace_bytes(h, n, 1) exceeds the array (for the DeepSeek-V3 shape
+ * that allows about 64 tokens per call). All calls share the one array, whose
+ * contents persist between calls: each call clears the device flag it holds
+ * (so the flag is not readable here), and calls that overlap on the GPU, on
+ * any streams, race. Calls no cudaMalloc, cudaFree or allocating routine. */
+int mla_decode_qkv_noalloc(mla_handle* h, const void* hidden, int n, const float* cos,
+                           const float* sin, void* kv_cache, int n_blocks,
+                           const int32_t* slot_mapping, void* q_abs, void* q_pe, void* stream);
+
 /* ---- prefill ------------------------------------------------------------------ */
 
 /* Causal prefill (context encoding) of one sequence of S tokens at positions
