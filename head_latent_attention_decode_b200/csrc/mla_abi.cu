@@ -429,26 +429,34 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
                                  (bf16*)(wsb + W.o_lat));
     return r != MLA_OK ? r : cuda_status();
   }
-  AttnArgs p{};
-  p.q_abs = q_abs; p.q_pe = q_pe; p.cache = kv_cache; p.n_blocks = n_blocks; p.bs = c->block_size;
-  p.block_table = block_table; p.mbps = max_blocks_per_seq; p.ctx = context_lens; p.max_ctx = max_context_len;
-  p.H = H; p.r_kv = rkv; p.d_r = dr; p.layout = c->row_layout; p.scale = h->scale;
-  p.n_splits = W.splits;
-  p.chunk = (int)cdiv(cdiv(max_context_len, W.splits), ATT_TR) * ATT_TR;
-  p.part_o = (float*)(wsb + W.part_o); p.part_ml = (float*)(wsb + W.part_ml); p.flag = flag;
-  const int R = rkv + dr;
-  const size_t smem = (size_t)(ATT_TR * (R + 1) + ATT_HPB * R) * 4;
-  dim3 grid(W.splits, n, (unsigned)cdiv(H, ATT_HPB));
-  mla_timer_begin("attn", s);
-  if (ta == 0) { set_smem(attn_decode_simt_kernel<float>, smem); attn_decode_simt_kernel<float><<<grid, 256, smem, s>>>(p); }
-  else { set_smem(attn_decode_simt_kernel<bf16>, smem); attn_decode_simt_kernel<bf16><<<grid, 256, smem, s>>>(p); }
-  mla_timer_end("attn", s);
-  count_launch();
   void* o_lat = wsb + W.o_lat;
-  dim3 cg(n, H);
-  if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat);
-  else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat);
-  count_launch();
+  if (tc_attention_supported(h)) {
+    // tensor-core attention (bf16 activations) ahead of CUDA-core W_UV / o_proj
+    const int r = tc_attention_core(h, q_abs, q_pe, kv_cache, n_blocks, block_table, max_blocks_per_seq,
+                                    context_lens, max_context_len, n, (float*)(wsb + W.part_o),
+                                    (float*)(wsb + W.part_ml), W.splits, (bf16*)o_lat, flag, s);
+    if (r != MLA_OK) return r;
+  } else {
+    AttnArgs p{};
+    p.q_abs = q_abs; p.q_pe = q_pe; p.cache = kv_cache; p.n_blocks = n_blocks; p.bs = c->block_size;
+    p.block_table = block_table; p.mbps = max_blocks_per_seq; p.ctx = context_lens; p.max_ctx = max_context_len;
+    p.H = H; p.r_kv = rkv; p.d_r = dr; p.layout = c->row_layout; p.scale = h->scale;
+    p.n_splits = W.splits;
+    p.chunk = (int)cdiv(cdiv(max_context_len, W.splits), ATT_TR) * ATT_TR;
+    p.part_o = (float*)(wsb + W.part_o); p.part_ml = (float*)(wsb + W.part_ml); p.flag = flag;
+    const int R = rkv + dr;
+    const size_t smem = (size_t)(ATT_TR * (R + 1) + ATT_HPB * R) * 4;
+    dim3 grid(W.splits, n, (unsigned)cdiv(H, ATT_HPB));
+    mla_timer_begin("attn", s);
+    if (ta == 0) { set_smem(attn_decode_simt_kernel<float>, smem); attn_decode_simt_kernel<float><<<grid, 256, smem, s>>>(p); }
+    else { set_smem(attn_decode_simt_kernel<bf16>, smem); attn_decode_simt_kernel<bf16><<<grid, 256, smem, s>>>(p); }
+    mla_timer_end("attn", s);
+    count_launch();
+    dim3 cg(n, H);
+    if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat);
+    else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat);
+    count_launch();
+  }
   // head_out[h] = o_lat[h] @ W_UV[h]
   LinearArgs a = lin(o_lat, (long long)H * rkv, h->base + L.Wuv, rkv, wscale(h, L.sWuv), cdiv(rkv, 128), head,
                      (long long)H * dv, n, dv, rkv);

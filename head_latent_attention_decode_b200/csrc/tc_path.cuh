@@ -10,6 +10,7 @@
 #include "simt_kernels.cuh"
 #include "tc_gemm.cuh"
 #include "tc_attn.cuh"
+#include "tc_attn_small.cuh"
 #include "tc_prefill_attn.cuh"
 
 namespace mla {
@@ -234,11 +235,13 @@ static inline size_t tc_decode_ws_bytes(const mla_handle* h, long long n, int) {
 static inline int tc_init(mla_handle* h) {
   TcState& T = h->tc;
   T.enabled = 0;
+  T.attn = 0;
   int dev = 0, major = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   cudaDeviceGetAttribute(&T.num_sms, cudaDevAttrMultiProcessorCount, dev);
   const mla_config& c = h->cfg;
+  T.attn = (major == 10 && c.act_dtype == MLA_BF16) ? 1 : 0;
   if (major != 10 || c.act_dtype != MLA_BF16 || c.weight_dtype != MLA_BF16) return MLA_OK;
   if (c.hidden % 64 || c.kv_lora_rank % 64 || c.qk_nope % 64 || c.q_lora_rank % 64 ||
       ((long long)c.n_heads * c.v_dim) % 64 || (c.qk_nope + c.qk_rope) % 2)
@@ -265,6 +268,7 @@ static inline int tc_init(mla_handle* h) {
 
 static inline bool tc_decode_qkv_supported(const mla_handle* h, int n) { return h->tc.enabled && n <= 256; }
 static inline bool tc_decode_attn_supported(const mla_handle* h, int n, int) { return h->tc.enabled && n <= 256; }
+static inline bool tc_attention_supported(const mla_handle* h) { return h->tc.attn != 0; }
 static inline bool tc_prefill_supported(const mla_handle* h, int) { return h->tc.enabled; }
 
 static GemmArgs gemm_args(int M, int N, int K, int batches, int mode, void* out, long long ldo, long long bstride,
@@ -323,23 +327,71 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   return launch_gemm(T.a_Wuk, mn, g3, bn, 1, T.num_sms, s);
 }
 
-static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const void* q_pe, const void* kv_cache,
-                                 int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
-                                 int max_ctx, int n, void* out, void* head, char* ws, size_t tc_off,
-                                 cudaStream_t s, float* part_o, float* part_ml, int splits, bf16* o_lat) {
+// Split-KV absorbed attention and the LSE merge of the splits -> o_lat (bf16).
+// tcgen05 kernel for the DeepSeek latent dims, CUDA-core kernel otherwise.
+static inline int tc_attention_core(const mla_handle* h, const void* q_abs, const void* q_pe, const void* kv_cache,
+                                    int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
+                                    int max_ctx, int n, float* part_o, float* part_ml, int splits, bf16* o_lat,
+                                    int* flag, cudaStream_t s) {
   const mla_config& c = h->cfg;
   const TcState& T = h->tc;
-  const TcDecodeWs W = tc_decode_ws(h, n);
-  char* tw = ws + tc_off;
-  int* flag = (int*)ws;
-  const int H = c.n_heads, dr = c.qk_rope, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
-  const int bn = pick_bn(n);
+  const int H = c.n_heads, dr = c.qk_rope, rkv = c.kv_lora_rank;
   int st;
   // 1. split-KV absorbed attention and the LSE merge -> o_lat (bf16)
   const int R = rkv + dr;
-  const bool tc_attn = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && H <= 128 &&
-                       (((uintptr_t)q_abs) & 15) == 0;
-  if (tc_attn) {
+  const bool latent_ok = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && (((uintptr_t)q_abs) & 15) == 0 &&
+                         (((uintptr_t)q_pe) & 15) == 0;
+  if (latent_ok && H <= 32) {
+    // few heads: transposed tiles, one CTA per (sequence, split). Pick the
+    // split length (whole 128-row tiles) that minimises waves x tiles per CTA.
+    const int sms = T.num_sms > 0 ? T.num_sms : 148;
+    const int tiles = (int)cdiv(max_ctx, 128);
+    int best_ct = tiles, best_cost = 1 << 30;
+    for (int ct = 1; ct <= tiles; ++ct) {
+      const int spl = (int)cdiv(tiles, ct);
+      if (spl > splits) continue;
+      const int waves = (int)cdiv((long long)n * spl, sms);
+      const int cost = waves * (ct + 2);   // + per-CTA set-up, in tiles
+      if (cost < best_cost) { best_cost = cost; best_ct = ct; }
+    }
+    const int chunk = best_ct * 128;
+    const int sp = (int)cdiv(max_ctx, chunk);
+    splits = sp;
+    const int NH = H <= 16 ? 16 : 32;
+    CUtensorMap mqa, mqp, mc;
+    if ((st = make_map2(&mqa, q_abs, rkv, (long long)n * H, rkv, NH)) != MLA_OK) return st;
+    if ((st = make_map2(&mqp, q_pe, dr, (long long)n * H, dr, NH)) != MLA_OK) return st;
+    if ((st = make_map2(&mc, kv_cache, R, (long long)n_blocks * c.block_size, R, 64)) != MLA_OK) return st;
+    TcAttnArgs ta{};
+    ta.n = n; ta.H = H; ta.splits = sp; ta.chunk = chunk;
+    ta.bs = c.block_size; ta.n_blocks = n_blocks; ta.mbps = mbps; ta.max_ctx = max_ctx;
+    ta.block_table = block_table; ta.ctx = ctx; ta.q_abs = (const bf16*)q_abs;
+    ta.lat_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? 0 : dr;
+    ta.rope_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? rkv : 0;
+    ta.scale_log2 = h->scale * 1.4426950408889634f;
+    ta.part_o = part_o; ta.part_ml = part_ml; ta.flag = flag;
+    static bool attr16[64] = {false}, attr32[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    mla_timer_begin("attn", s);
+    if (NH == 16) {
+      if (dev < 64 && !attr16[dev]) {
+        cudaFuncSetAttribute(tc_attn_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnSmallSmem<16>::SIZE);
+        attr16[dev] = true;
+      }
+      tc_attn_small_kernel<16><<<n * sp, 192, AttnSmallSmem<16>::SIZE, s>>>(mqa, mqp, mc, ta);
+    } else {
+      if (dev < 64 && !attr32[dev]) {
+        cudaFuncSetAttribute(tc_attn_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnSmallSmem<32>::SIZE);
+        attr32[dev] = true;
+      }
+      tc_attn_small_kernel<32><<<n * sp, 192, AttnSmallSmem<32>::SIZE, s>>>(mqa, mqp, mc, ta);
+    }
+    mla_timer_end("attn", s);
+    mla_count_launch(1);
+  } else if (latent_ok && H <= 128) {
     // (sequence, split) clusters: about three waves of CTA pairs, at most the
     // splits the workspace holds
     const int pairs = T.num_sms / 2 > 0 ? T.num_sms / 2 : 74;
@@ -387,6 +439,23 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   }
   attn_combine_kernel<bf16><<<dim3(n, H), 128, 0, s>>>(part_o, part_ml, splits, H, rkv, o_lat);
   mla_count_launch(1);
+  return MLA_OK;
+}
+
+static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const void* q_pe, const void* kv_cache,
+                                 int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
+                                 int max_ctx, int n, void* out, void* head, char* ws, size_t tc_off,
+                                 cudaStream_t s, float* part_o, float* part_ml, int splits, bf16* o_lat) {
+  const mla_config& c = h->cfg;
+  const TcState& T = h->tc;
+  const TcDecodeWs W = tc_decode_ws(h, n);
+  char* tw = ws + tc_off;
+  int* flag = (int*)ws;
+  const int H = c.n_heads, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
+  const int bn = pick_bn(n);
+  int st = tc_attention_core(h, q_abs, q_pe, kv_cache, n_blocks, block_table, mbps, ctx, max_ctx, n, part_o,
+                             part_ml, splits, o_lat, flag, s);
+  if (st != MLA_OK) return st;
   // 2. head_out[h] = o_lat[h] @ W_UV[h]  (A = Wuv[h] [d_v, r_kv], B = o_lat[:, h, :])
   CUtensorMap mo;
   if ((st = make_map(&mo, o_lat, rkv, H, n, (long long)rkv * 2, (long long)H * rkv * 2, bn, 1)) != MLA_OK) return st;

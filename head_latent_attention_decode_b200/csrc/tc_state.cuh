@@ -5,7 +5,8 @@
 #include <cuda.h>
 
 struct TcState {
-  int enabled;       // bf16 activations with bf16 weights on an sm_100 device
+  int enabled;       // bf16 activations with bf16 weights on an sm_100 device (all tcgen05 GEMMs)
+  int attn;          // bf16 activations on an sm_100 device (tcgen05 attention, any weight dtype)
   int num_sms;
   // weights as the A operand (decode, swap-AB): 128-row boxes
   CUtensorMap a_W1, a_Wqb, a_Wuk, a_Wuv, a_Wo;
