@@ -9,6 +9,7 @@
 #include "handle.cuh"
 #include "simt_kernels.cuh"
 #include "tc_gemm.cuh"
+#include "tc_gemm_fp8.cuh"
 #include "tc_attn.cuh"
 #include "tc_attn_small.cuh"
 #include "tc_prefill_attn.cuh"
@@ -37,15 +38,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 64 K-elements x `box_rows` rows; the rows are dimension 1 (rows_dim2 = 0) or
 // dimension 2 (rows_dim2 = 1). Strides in bytes. Out-of-range elements read 0.
 static int make_map(CUtensorMap* m, const void* base, long long K, long long d1, long long d2, long long s1,
-                    long long s2, int box_rows, int rows_dim2) {
+                    long long s2, int box_rows, int rows_dim2, bool u8 = false) {
   auto fn = encode_fn();
   if (!fn) return MLA_ERR_CUDA;
   if (((uintptr_t)base) & 15 || s1 % 16 || s2 % 16) return MLA_ERR_UNSUPPORTED;
   cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)d1, (cuuint64_t)d2};
   cuuint64_t strides[2] = {(cuuint64_t)s1, (cuuint64_t)s2};
-  cuuint32_t box[3] = {64, (cuuint32_t)(rows_dim2 ? 1 : box_rows), (cuuint32_t)(rows_dim2 ? box_rows : 1)};
+  // 128-byte rows: 64 bf16 or 128 FP8 codes
+  cuuint32_t box[3] = {(cuuint32_t)(u8 ? 128 : 64), (cuuint32_t)(rows_dim2 ? 1 : box_rows),
+                       (cuuint32_t)(rows_dim2 ? box_rows : 1)};
   cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
@@ -99,6 +103,46 @@ static int launch_gemm(const CUtensorMap& A, const CUtensorMap& B, GemmArgs g, i
     case 64: return launch_gemm_bn<64>(A, B, g, num_sms, s);
     case 128: return launch_gemm_bn<128>(A, B, g, num_sms, s);
     default: return launch_gemm_bn<256>(A, B, g, num_sms, s);
+  }
+}
+
+template <int BN>
+static int launch_gemm_fp8_bn(const CUtensorMap& A, const CUtensorMap& B, const Fp8GemmArgs& fa, int num_sms,
+                              cudaStream_t s) {
+  using C = Fp8Cfg<BN>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaFuncSetAttribute(tc_gemm_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    attr_set[dev] = true;
+  }
+  const int grid = fa.g.total_units < num_sms ? fa.g.total_units : num_sms;
+  tc_gemm_fp8_kernel<BN><<<grid, 192, C::SMEM, s>>>(A, B, fa);
+  mla_count_launch(1);
+  return MLA_OK;
+}
+
+// FP8-weight GEMM (A = codes, K blocks of 128 = one scale column each).
+static int launch_gemm_fp8(const CUtensorMap& A, const CUtensorMap& B, GemmArgs g, int bn, int splits,
+                           const float* scale, long long scale_ld, long long scale_batch, int num_sms,
+                           cudaStream_t s) {
+  g.m_tiles = (int)cdiv(g.M, 128);
+  g.n_tiles = (int)cdiv(g.N, bn);
+  g.k_blocks = (int)cdiv(g.K, 128);
+  if (splits < 1) splits = 1;
+  if (splits > g.k_blocks) splits = g.k_blocks;
+  g.kb_per_split = (int)cdiv(g.k_blocks, splits);
+  g.splits = (int)cdiv(g.k_blocks, g.kb_per_split);
+  g.total_units = g.m_tiles * g.n_tiles * g.batches * g.splits;
+  if (g.total_units <= 0) return MLA_OK;
+  Fp8GemmArgs fa{};
+  fa.g = g; fa.scale = scale; fa.scale_ld = scale_ld; fa.scale_batch = scale_batch;
+  switch (bn) {
+    case 16: return launch_gemm_fp8_bn<16>(A, B, fa, num_sms, s);
+    case 32: return launch_gemm_fp8_bn<32>(A, B, fa, num_sms, s);
+    case 64: return launch_gemm_fp8_bn<64>(A, B, fa, num_sms, s);
+    default: return launch_gemm_fp8_bn<128>(A, B, fa, num_sms, s);
   }
 }
 
@@ -215,8 +259,9 @@ static TcDecodeWs tc_decode_ws(const mla_handle* h, long long n) {
   const mla_config& c = h->cfg;
   const WeightLayout& L = h->L;
   const int sms = h->tc.num_sms > 0 ? h->tc.num_sms : 148;
-  w.s1 = decode_splits_for((int)cdiv(L.N1, 128), (int)cdiv(c.hidden, 64), sms);
-  w.s5 = decode_splits_for((int)cdiv(c.hidden, 128), (int)cdiv((long long)c.n_heads * c.v_dim, 64), sms);
+  const int ku = h->tc.fp8 ? 128 : 64;   // K block of the GEMM kernel in use
+  w.s1 = decode_splits_for((int)cdiv(L.N1, 128), (int)cdiv(c.hidden, ku), sms);
+  w.s5 = decode_splits_for((int)cdiv(c.hidden, 128), (int)cdiv((long long)c.n_heads * c.v_dim, ku), sms);
   size_t off = 0;
   auto put = [&](size_t b) { size_t o = off; off = align_up(off + b, 256); return o; };
   w.Yp = put((size_t)w.s1 * n * L.N1 * 4);
@@ -228,7 +273,7 @@ static TcDecodeWs tc_decode_ws(const mla_handle* h, long long n) {
 }
 
 static inline size_t tc_decode_ws_bytes(const mla_handle* h, long long n, int) {
-  if (!h->tc.enabled) return 0;
+  if (!h->tc.enabled && !h->tc.fp8) return 0;
   return tc_decode_ws(h, n).total;
 }
 
@@ -236,12 +281,28 @@ static inline int tc_init(mla_handle* h) {
   TcState& T = h->tc;
   T.enabled = 0;
   T.attn = 0;
+  T.fp8 = 0;
   int dev = 0, major = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   cudaDeviceGetAttribute(&T.num_sms, cudaDevAttrMultiProcessorCount, dev);
   const mla_config& c = h->cfg;
   T.attn = (major == 10 && c.act_dtype == MLA_BF16) ? 1 : 0;
+  if (major == 10 && c.act_dtype == MLA_BF16 && c.weight_dtype == MLA_FP8_E4M3_B128 && c.hidden % 128 == 0 &&
+      c.kv_lora_rank % 128 == 0 && ((long long)c.n_heads * c.v_dim) % 128 == 0 && (c.qk_nope + c.qk_rope) % 2 == 0) {
+    const WeightLayout& L = h->L;
+    const char* b = h->base;
+    const long long H = c.n_heads, dn = c.qk_nope, dv = c.v_dim, rkv = c.kv_lora_rank, D = c.hidden;
+    const long long rq = c.q_lora_rank;
+    int st = MLA_OK;
+    st |= make_map(&T.a8_W1, b + L.W1, D, L.N1, 1, D, D * L.N1, 128, 0, true);
+    if (rq) st |= make_map(&T.a8_Wqb, b + L.Wqb, rq, L.Hq, 1, rq, rq * L.Hq, 128, 0, true);
+    st |= make_map(&T.a8_Wuk, b + L.Wuk, dn, rkv, H, dn, rkv * dn, 128, 0, true);
+    st |= make_map(&T.a8_Wuv, b + L.Wuv, rkv, dv, H, rkv, dv * rkv, 128, 0, true);
+    st |= make_map(&T.a8_Wo, b + L.Wo, H * dv, D, 1, H * dv, H * dv * D, 128, 0, true);
+    if (st == MLA_OK) T.fp8 = 1;
+    return MLA_OK;
+  }
   if (major != 10 || c.act_dtype != MLA_BF16 || c.weight_dtype != MLA_BF16) return MLA_OK;
   if (c.hidden % 64 || c.kv_lora_rank % 64 || c.qk_nope % 64 || c.q_lora_rank % 64 ||
       ((long long)c.n_heads * c.v_dim) % 64 || (c.qk_nope + c.qk_rope) % 2)
@@ -266,8 +327,40 @@ static inline int tc_init(mla_handle* h) {
   return MLA_OK;
 }
 
-static inline bool tc_decode_qkv_supported(const mla_handle* h, int n) { return h->tc.enabled && n <= 256; }
-static inline bool tc_decode_attn_supported(const mla_handle* h, int n, int) { return h->tc.enabled && n <= 256; }
+static inline bool tc_decode_qkv_supported(const mla_handle* h, int n) {
+  return (h->tc.enabled && n <= 256) || (h->tc.fp8 && n <= 128);
+}
+static inline bool tc_decode_attn_supported(const mla_handle* h, int n, int) {
+  return (h->tc.enabled && n <= 256) || (h->tc.fp8 && n <= 128);
+}
+
+enum WSel { W_1, W_QB, W_UK, W_UV, W_O };
+
+// Weight GEMM of the decode path: bf16 weights on tc_gemm_kernel, FP8 weights
+// on tc_gemm_fp8_kernel with the matrix's block scales.
+static int wgemm(const mla_handle* h, WSel w, const CUtensorMap& B, GemmArgs g, int bn, int splits, cudaStream_t s) {
+  const TcState& T = h->tc;
+  if (!T.fp8) {
+    const CUtensorMap* A = w == W_1 ? &T.a_W1 : w == W_QB ? &T.a_Wqb : w == W_UK ? &T.a_Wuk : w == W_UV ? &T.a_Wuv : &T.a_Wo;
+    return launch_gemm(*A, B, g, bn, splits, T.num_sms, s);
+  }
+  const WeightLayout& L = h->L;
+  const mla_config& c = h->cfg;
+  const char* base = h->base;
+  const long long D = c.hidden, rq = c.q_lora_rank, dn = c.qk_nope, dv = c.v_dim, rkv = c.kv_lora_rank;
+  const long long H = c.n_heads;
+  const CUtensorMap* A;
+  const float* sc;
+  long long ld, bs = 0;
+  switch (w) {
+    case W_1: A = &T.a8_W1; sc = (const float*)(base + L.sW1); ld = cdiv(D, 128); break;
+    case W_QB: A = &T.a8_Wqb; sc = (const float*)(base + L.sWqb); ld = cdiv(rq, 128); break;
+    case W_UK: A = &T.a8_Wuk; sc = (const float*)(base + L.sWuk); ld = cdiv(dn, 128); bs = cdiv(rkv, 128) * ld; break;
+    case W_UV: A = &T.a8_Wuv; sc = (const float*)(base + L.sWuv); ld = cdiv(rkv, 128); bs = cdiv(dv, 128) * ld; break;
+    default: A = &T.a8_Wo; sc = (const float*)(base + L.sWo); ld = cdiv(H * dv, 128); break;
+  }
+  return launch_gemm_fp8(*A, B, g, bn, splits, sc, ld, bs, T.num_sms, s);
+}
 static inline bool tc_attention_supported(const mla_handle* h) { return h->tc.attn != 0; }
 static inline bool tc_prefill_supported(const mla_handle* h, int) { return h->tc.enabled; }
 
@@ -295,7 +388,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   CUtensorMap mx;
   if ((st = make_map2(&mx, hidden, D, n, D, bn)) != MLA_OK) return st;
   GemmArgs g = gemm_args(L.N1, n, D, 1, EPI_F32_T, tw + W.Yp, L.N1, 0, flag);
-  if ((st = launch_gemm(T.a_W1, mx, g, bn, W.s1, T.num_sms, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_1, mx, g, bn, W.s1, s)) != MLA_OK) return st;
   // 2. split sum, norms, RoPE, scatter (and, without q_lora, q_nope / q_pe)
   FrontFoldTcArgs f{};
   f.Yp = (const float*)(tw + W.Yp); f.split_stride = (long long)n * L.N1; f.splits = W.s1; f.N1 = L.N1;
@@ -316,7 +409,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
     if ((st = make_map2(&mq, tw + W.qn, rq, n, rq, bn)) != MLA_OK) return st;
     GemmArgs g2 = gemm_args(L.Hq, n, rq, 1, EPI_QROPE_T, tw + W.q_nope, 0, 0, flag);
     g2.out2 = q_pe; g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr;
-    if ((st = launch_gemm(T.a_Wqb, mq, g2, bn, 1, T.num_sms, s)) != MLA_OK) return st;
+    if ((st = wgemm(h, W_QB, mq, g2, bn, 1, s)) != MLA_OK) return st;
   }
   // 4. q_abs[h] = q_nope[h] @ W_UK[h]  (batched over heads: A = Wuk[h] [r_kv, d_n], B = q_nope[:, h, :])
   CUtensorMap mn;
@@ -324,7 +417,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
     return st;
   GemmArgs g3 = gemm_args(rkv, n, dn, H, EPI_BF16_T, q_abs, (long long)H * rkv, rkv, flag);
   g3.b_rows_dim2 = 1;
-  return launch_gemm(T.a_Wuk, mn, g3, bn, 1, T.num_sms, s);
+  return wgemm(h, W_UK, mn, g3, bn, 1, s);
 }
 
 // Split-KV absorbed attention and the LSE merge of the splits -> o_lat (bf16).
@@ -461,12 +554,12 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   if ((st = make_map(&mo, o_lat, rkv, H, n, (long long)rkv * 2, (long long)H * rkv * 2, bn, 1)) != MLA_OK) return st;
   GemmArgs g4 = gemm_args(dv, n, rkv, H, EPI_BF16_T, head, (long long)H * dv, dv, flag);
   g4.b_rows_dim2 = 1;
-  if ((st = launch_gemm(T.a_Wuv, mo, g4, bn, 1, T.num_sms, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_UV, mo, g4, bn, 1, s)) != MLA_OK) return st;
   // 3. out = head_out @ wo  (swap-AB, K split, then reduce to bf16)
   CUtensorMap mh;
   if ((st = make_map2(&mh, head, (long long)H * dv, n, (long long)H * dv, bn)) != MLA_OK) return st;
   GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
-  if ((st = launch_gemm(T.a_Wo, mh, g5, bn, W.s5, T.num_sms, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_O, mh, g5, bn, W.s5, s)) != MLA_OK) return st;
   const long long cnt = (long long)n * D;
   splitk_reduce_bf16_kernel<<<(unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s>>>(
       (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);
