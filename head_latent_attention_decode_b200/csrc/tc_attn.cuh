@@ -16,8 +16,10 @@
 //                                          N 256, K 64; V = the same shared-memory
 //                                          tile read MN-major)
 // Every cache byte is read from HBM once, O (128 x 512 fp32) is split over the
-// two CTAs' TMEM, and a 4-deep ring of tiles keeps loads in flight while the
-// MMA thread issues S of later tiles ahead of P.V of earlier ones. Partials
+// two CTAs' TMEM, and a 3-deep ring of tiles keeps loads in flight while the
+// MMA thread issues S of later tiles ahead of P.V of earlier ones. Warps 0-3
+// run the softmax, warps 6-9 send each tile's partial scores to the peer as
+// soon as S lands, warp 4 issues TMA and warp 5 the MMAs. Partials
 // (unnormalised O, reference max, sum) go to the workspace and
 // attn_combine_kernel merges the splits.
 #pragma once
@@ -40,7 +42,9 @@ struct TcAttnArgs {
   int* flag;
   // optional tracing: %globaltimer stamps of cluster 0, CTA 0, for its first 64
   // tiles, [tile][16]: softmax (head 0) 0 iteration start, 2 peer partial
-  // arrived, 3 scores summed, 4 P computed, 5 P handed over, 1 next partial sent;
+  // arrived, 6 S ready, 7 S read, 11 partials added, 3 peer buffer freed,
+  // 4 P computed, 5 P handed over; sender (head 0) 12 S ready, 13 S read,
+  // 14 peer buffer free, 1 partial sent;
   // 8 S issued, 9 P.V issued (MMA thread); 10 tile load issued (producer);
   // [0][15] unit start. NULL = off.
   unsigned long long* trace;
@@ -51,8 +55,9 @@ struct AttnSmem {
   static constexpr int STAGE = 5 * 8192;        // 4 latent + 1 rope slot of [64 rows x 64 cols] bf16
   static constexpr int TILE_OFF = 0;
   static constexpr int QR_OFF = ATT_NST * STAGE;  // q_pe [128 x 64] bf16 (CTA 0)
-  static constexpr int X_OFF = QR_OFF + 16384;    // 2 x [128 x 64] fp32, the peer's partial S
-  static constexpr int BAR_OFF = X_OFF + 2 * 32768;
+  static constexpr int X_OFF = QR_OFF + 16384;    // [128 x 64] fp32, the peer's partial S
+  static constexpr int STG_OFF = X_OFF + 32768;   // [128 x 64] fp32, our partial on its way out
+  static constexpr int BAR_OFF = STG_OFF + 32768;
   static constexpr int SIZE = 1024 + BAR_OFF + 256;
 };
 // TMEM columns: Q latent [0,128) (bf16 pairs), S/P buffers [128,192) [192,256), O [256,512)
@@ -68,7 +73,7 @@ __device__ __forceinline__ int attn_tile_rows(const TcAttnArgs& a, int b, int j0
   return min(64, r1 - j0);
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_qpe, const __grid_constant__ CUtensorMap tm_cache,
                           TcAttnArgs a) {
   using SM = AttnSmem;
@@ -84,7 +89,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const uint32_t p_full_b = s_full_b + 16;             // [2]
   const uint32_t sp_empty_b = p_full_b + 16;           // [2] S/P buffer free (P.V done)
   const uint32_t q_ready = sp_empty_b + 16, qr_full = q_ready + 8, o_done = qr_full + 8;
-  const uint32_t x_full_b = o_done + 8, x_free_b = x_full_b + 16, fin = x_free_b + 16;   // x_*: [2]
+  const uint32_t x_full_b = o_done + 8, x_free_b = x_full_b + 16, fin = x_free_b + 16;   // x_full, x_free
+  const uint32_t s_read_b = fin + 8;   // [2] the sender has read S(t) out of TMEM
   uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 192);
   volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 196);
 
@@ -121,7 +127,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     mbar_init(q_ready, 128);
     mbar_init(qr_full, 1);
     mbar_init(o_done, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(x_full_b + 8 * i, 1); mbar_init(x_free_b + 8 * i, 4); }
+    mbar_init(x_full_b, 1);
+    mbar_init(x_free_b, 4);
+    for (int i = 0; i < 2; ++i) mbar_init(s_read_b + 8 * i, 128);
     mbar_init(fin, 1);
     *abort_word = 0;
     fence_mbar_init();
@@ -232,6 +240,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       while (!mbar_try_wait(fin, 0))
         if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
     }
+  } else if (warp >= 6) {
+    // ---------------- senders: S_r(k) -> staging -> one bulk copy into the peer's X ----------------
+    const int h = 32 * (warp & 3) + lane;                 // TMEM lane quarter of this warp
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const bool issuer = (warp == 6 && lane == 0);
+    const uint32_t peer_x = mapa_shared(x_s, peer), peer_x_full = mapa_shared(x_full_b, peer);
+    const uint32_t stg_s = sbase + SM::STG_OFF;
+    float4* stg_row = (float4*)(smem + SM::STG_OFF + h * 256);
+    for (int k = 0; k < T; ++k) {
+      const int kb = k & 1;
+      if (!mbar_wait_warp(s_full_b + 8 * kb, (k >> 1) & 1, abort_word, a.flag)) break;
+      const bool trs = a.trace && cid == 0 && r == 0 && h == 0 && k < 64;
+      if (trs) a.trace[k * 16 + 12] = global_timer_ns();
+      tc_fence_after();
+      float v[64];
+      const uint32_t sa = tmem + ATT_TM_S + 64 * kb + lane_base;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld16(sa + 16 * c, (uint32_t*)&v[16 * c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(s_read_b + 8 * kb);
+      if (trs) a.trace[k * 16 + 13] = global_timer_ns();
+      if (issuer) bulk_wait_read_all();                  // the previous copy has left the staging buffer
+      named_bar_sync(2, 128);
+#pragma unroll
+      for (int c = 0; c < 16; ++c)   // chunk c of row h at slot c ^ (h & 15): no bank conflicts
+        stg_row[c ^ (h & 15)] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      fence_proxy_async_smem();
+      named_bar_sync(2, 128);
+      if (issuer) {
+        // the peer has consumed what we sent for tile k - 1
+        bool ok = mbar_wait_cluster(x_free_b, (k & 1) ^ 1, abort_word, a.flag);
+        if (trs) a.trace[k * 16 + 14] = global_timer_ns();
+        if (ok) {
+          bulk_copy_to_peer(peer_x, stg_s, 32768, peer_x_full);
+          bulk_commit_group();
+        }
+      }
+      if (trs) a.trace[k * 16 + 1] = global_timer_ns();
+    }
+    if (issuer) bulk_wait_read_all();
   } else {
     // ---------------- softmax: thread h <-> head h <-> TMEM lane h ----------------
     const int h = threadIdx.x;
@@ -253,29 +302,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(q_ready);
     }
-    // partial-score exchange: S_r(k) goes with st.async into the peer's X[k & 1],
-    // completing bytes on the peer's x_full[k & 1]; each peer warp frees the
-    // buffer with one remote arrive on our x_free[k & 1] once it has read it.
-    const uint32_t peer_x = mapa_shared(x_s + h * 256, peer);
-    const uint32_t peer_x_full = mapa_shared(x_full_b, peer), peer_x_free = mapa_shared(x_free_b, peer);
-    float v[64];   // own partial of the tile processed next (already sent to the peer)
-    auto load_and_send = [&](int k) -> bool {
-      const int kb = k & 1;
-      if (!mbar_wait_warp(s_full_b + 8 * kb, (k >> 1) & 1, abort_word, a.flag)) return false;
-      tc_fence_after();
-      const uint32_t sa = tmem + ATT_TM_S + 64 * kb + lane_base;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(sa + 16 * c, (uint32_t*)&v[16 * c]);
-      tmem_ld_wait();
-      if (!mbar_wait_cluster_warp(x_free_b + 8 * kb, ((k >> 1) & 1) ^ 1, abort_word, a.flag)) return false;
-      const uint32_t dst = peer_x + kb * 32768, bar_k = peer_x_full + 8 * kb;
-#pragma unroll
-      for (int c = 0; c < 16; ++c)   // chunk c of row h at slot c ^ (h & 15): no bank conflicts
-        st_async_v4(dst + 16 * (c ^ (h & 15)), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3], bar_k);
-      return true;
-    };
+    const uint32_t peer_x_free = mapa_shared(x_free_b, peer);
     float m_ref = -INFINITY, l = 0.f;
-    bool ok = load_and_send(0);
+    bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int sb = t & 1, st = t % ATT_NST;
       long long row_unused;
@@ -283,23 +312,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       if (valid < 0) valid = 0;
       const bool tr = trace && h == 0 && t < 64;
       if (tr) trace[t * 16 + 0] = global_timer_ns();
-      if (h == 0) mbar_arrive_expect_tx(x_full_b + 8 * sb, 32768);
-      if (!mbar_wait_warp(x_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (h == 0) mbar_arrive_expect_tx(x_full_b, 32768);
+      if (!mbar_wait_warp(x_full_b, t & 1, abort_word, a.flag)) { ok = false; break; }
       if (tr) trace[t * 16 + 2] = global_timer_ns();
-      const float4* xloc = (const float4*)(smem + SM::X_OFF + sb * 32768 + h * 256);
+      if (!mbar_wait_warp(s_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (tr) trace[t * 16 + 6] = global_timer_ns();
+      tc_fence_after();
+      float v[64];
+      const uint32_t sp_addr = tmem + ATT_TM_S + 64 * sb + lane_base;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld16(sp_addr + 16 * c, (uint32_t*)&v[16 * c]);
+      tmem_ld_wait();
+      if (tr) trace[t * 16 + 7] = global_timer_ns();
+      const float4* xloc = (const float4*)(smem + SM::X_OFF + h * 256);
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const float4 x = xloc[c ^ (h & 15)];
         v[4 * c] += x.x; v[4 * c + 1] += x.y; v[4 * c + 2] += x.z; v[4 * c + 3] += x.w;
       }
+      if (tr) trace[t * 16 + 11] = global_timer_ns();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(peer_x_free + 8 * sb);
+      if (lane == 0) mbar_arrive_remote_relaxed(peer_x_free);
       if (tr) trace[t * 16 + 3] = global_timer_ns();
       // online softmax in log2 units with a lazily moved reference max
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < 64; ++j)
-        if (j < valid) m4[j & 3] = fmaxf(m4[j & 3], v[j]);
+      for (int j = 0; j < 64; ++j) {
+        v[j] = (j < valid) ? v[j] : -INFINITY;          // also drops NaN from rows past the context
+        m4[j & 3] = fmaxf(m4[j & 3], v[j]);
+      }
       const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -312,10 +353,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
-        const float p0 = (j < valid) ? ex2_approx(fmaf(v[j], a.scale_log2, nm)) : 0.f;
-        const float p1 = (j + 1 < valid) ? ex2_approx(fmaf(v[j + 1], a.scale_log2, nm)) : 0.f;
-        __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        ps[(j >> 1) & 3] += __low2float(pb) + __high2float(pb);
+        __nv_bfloat162 pb = __floats2bfloat162_rn(ex2_approx(fmaf(v[j], a.scale_log2, nm)),
+                                                  ex2_approx(fmaf(v[j + 1], a.scale_log2, nm)));
+        const float2 pf = __bfloat1622float2(pb);
+        ps[(j >> 1) & 3] += pf.x + pf.y;
         pk[j >> 1] = *reinterpret_cast<uint32_t*>(&pb);
       }
       const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
@@ -345,15 +386,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
         fence_proxy_async_smem();
       }
-      const uint32_t sp_addr = tmem + ATT_TM_S + 64 * sb + lane_base;
+      // the sender must have read S(t) before P overwrites it
+      if (!mbar_wait_warp(s_read_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       tmem_st16(sp_addr, pk);            // P over S: 32 columns of bf16 pairs
       tmem_st16(sp_addr + 16, pk + 16);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full_b + 8 * sb);
       if (tr) trace[t * 16 + 5] = global_timer_ns();
-      if (t + 1 < T && !load_and_send(t + 1)) { ok = false; break; }
-      if (tr) trace[t * 16 + 1] = global_timer_ns();
     }
     if (ok && mbar_wait_warp(o_done, (T - 1) & 1, abort_word, a.flag)) {
       tc_fence_after();

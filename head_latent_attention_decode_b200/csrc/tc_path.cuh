@@ -513,7 +513,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
       attr[dev] = true;
     }
     mla_timer_begin("attn", s);
-    tc_attn_decode_kernel<<<2 * n * sp, 192, AttnSmem::SIZE, s>>>(mqp, mc, ta);
+    tc_attn_decode_kernel<<<2 * n * sp, 320, AttnSmem::SIZE, s>>>(mqp, mc, ta);
     mla_timer_end("attn", s);
     mla_count_launch(1);
   } else {
