@@ -87,6 +87,42 @@ def prefill_flops(s: wl.MlaShape, S: int) -> dict:
 
 
 # ---------------------------------------------------------------------------
+# DRAM traffic of the dominant kernel, from the committed ncu summary
+# ---------------------------------------------------------------------------
+
+KERNEL_SOURCES = {
+    "tc_attn_decode_kernel": "tc_attn.cuh",
+    "tc_attn_small_kernel": "tc_attn_small.cuh",
+    "tc_prefill_attn_kernel": "tc_prefill_attn.cuh",
+}
+
+
+def dominant_kernel(w: wl.Workload) -> str:
+    if w.mode == "prefill":
+        return "tc_prefill_attn_kernel"
+    return "tc_attn_small_kernel" if w.shape.n_heads <= 32 else "tc_attn_decode_kernel"
+
+
+def measured_traffic(kernel: str, workload: str):
+    """dram read + write bytes per launch from profiles/ncu_<kernel>_<workload>.md,
+    or None when there is no capture or the kernel source changed since it."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"ncu_{kernel}_{workload}.md")
+    src = os.path.join(ROOT, "head_latent_attention_decode_b200", "csrc", KERNEL_SOURCES.get(kernel, ""))
+    if not os.path.exists(path) or not os.path.isfile(src):
+        return None
+    text = open(path).read()
+    m_b = re.search(r"dram bytes per launch: (\d+)", text)
+    m_h = re.search(r"kernel source sha256: ([0-9a-f]{64})", text)
+    if not m_b or not m_h:
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_h.group(1):
+        return None
+    return int(m_b.group(1))
+
+
+# ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
 
@@ -406,6 +442,7 @@ def run_ours(args, world, rank, local):
         # dominant kernel, timed live with event nodes around its launch
         kname = "attn" if w.mode == "decode" else "prefill_attn"
         kms = all_max(kernel_time(step, kname, max(3, args.steps), flush, stream), world)
+        kern = dominant_kernel(w) if torch.cuda.get_device_capability()[0] == 10 else kname
         # end to end through the C-ABI with host buffers
         h2d, d2h = step.e2e_setup()
         for _ in range(2):
@@ -429,10 +466,10 @@ def run_ours(args, world, rank, local):
         work = step.work
         value, unit = toks / (ms / 1e3), "tokens/s"
         achieved = work["attn_bytes"] / (kms / 1e3) / 1e9
-        roof = {"bound": "hbm", "kernel": "attn", "achieved": round(achieved, 1),
+        roof = {"bound": "hbm", "kernel": kern, "achieved": round(achieved, 1),
                 "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                 "peak_source": peak_src, "kernel_ms": round(kms, 4),
-                "algorithmic_bytes": work["attn_bytes"], "traffic": None}
+                "algorithmic_bytes": work["attn_bytes"], "traffic": measured_traffic(kern, w.name)}
         extra = {"step_hbm_gbs": round(work["step_bytes"] / (ms / 1e3) / 1e9, 1),
                  "step_hbm_frac": round(work["step_bytes"] / (ms / 1e3) / 1e9 / hbm_peak, 4),
                  "step_algorithmic_bytes": work["step_bytes"]}
@@ -448,10 +485,10 @@ def run_ours(args, world, rank, local):
         fl = step.flops
         value, unit = fl["total"] * world / (ms / 1e3) / 1e12, "TFLOP/s"
         achieved = fl["attn"] / (kms / 1e3) / 1e12
-        roof = {"bound": "tensor", "kernel": "prefill_attn", "achieved": round(achieved, 2),
+        roof = {"bound": "tensor", "kernel": kern, "achieved": round(achieved, 2),
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
                 "peak_source": peak_src, "kernel_ms": round(kms, 4),
-                "algorithmic_flops": fl["attn"], "traffic": None}
+                "algorithmic_flops": fl["attn"], "traffic": measured_traffic(kern, w.name)}
         extra = {"tokens_per_s": round(toks / (ms / 1e3), 1), "step_flops": fl["total"]}
         e2e_val = fl["total"] * world / (e2e / 1e3) / 1e12
         metric = METRIC_PREFILL

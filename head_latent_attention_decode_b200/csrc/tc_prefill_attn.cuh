@@ -3,7 +3,7 @@
 // K_h = [k_nope_h | k_pe] with the rotated k_pe shared by every head, V_h from
 // the value half of wkv_b's output).
 //
-// One CTA per (128-query tile, head). Per 128-key tile j <= the query tile:
+// One CTA per (128-query tile, head), head-major. Per 128-key tile j <= the query tile:
 //   S = Q_h . K_h^T           tcgen05, M 128 x N 128, K 192 (Q resident in smem)
 //   online softmax, one thread per query row, lazy rescale of O when the row
 //   max grows by more than 2^8; keys past the query (diagonal tile) and past
@@ -48,9 +48,11 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 128);
   volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 132);
 
-  // heaviest query tiles first (causal work grows with the tile index)
-  const int qt = a.q_tiles - 1 - (int)(blockIdx.x / a.H);
-  const int h = blockIdx.x % a.H;
+  // head-major order so that the CTAs in flight share one or two heads' K/V in
+  // L2; within a head the heaviest query tiles (causal work grows with the
+  // tile index) go first
+  const int h = (int)(blockIdx.x / a.q_tiles);
+  const int qt = a.q_tiles - 1 - (int)(blockIdx.x % a.q_tiles);
   const int T = qt + 1;                       // key tiles 0..qt
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
