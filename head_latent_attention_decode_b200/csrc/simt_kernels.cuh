@@ -298,32 +298,50 @@ __global__ void __launch_bounds__(256) attn_decode_simt_kernel(AttnArgs p) {
 }
 
 // Merge split partials: o_lat = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s.
-// grid (n, H). Writes o_lat [n, H, r_kv] in act dtype.
+// grid (n, H), 128 threads x 4 consecutive columns (r_kv <= 512, r_kv % 4 == 0).
+// Writes o_lat [n, H, r_kv] in act dtype.
 template <typename T>
-__global__ void attn_combine_kernel(const float* part_o, const float* part_ml, int n_splits, int H,
-                                    int r_kv, T* o_lat) {
+__global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, const float* part_ml, int n_splits,
+                                                           int H, int r_kv, T* o_lat) {
+  __shared__ float wsh[64];
+  __shared__ float inv_sh;
   const int t = blockIdx.x, h = blockIdx.y;
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) {
-    const long long base = ((long long)t * n_splits + s) * H + h;
-    if (part_ml[base * 2 + 1] > 0.f) M = fmaxf(M, part_ml[base * 2]);
-  }
-  float den = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    const long long base = ((long long)t * n_splits + s) * H + h;
-    const float l = part_ml[base * 2 + 1];
-    if (l > 0.f) den += __expf(part_ml[base * 2] - M) * l;
-  }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  for (int c = threadIdx.x; c < r_kv; c += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < n_splits; ++s) {
+  if (threadIdx.x < 32) {
+    float M = -INFINITY;
+    for (int s = threadIdx.x; s < n_splits; s += 32) {
+      const long long base = ((long long)t * n_splits + s) * H + h;
+      if (part_ml[base * 2 + 1] > 0.f) M = fmaxf(M, part_ml[base * 2]);
+    }
+    M = warp_max(M);
+    float den = 0.f;
+    for (int s = threadIdx.x; s < n_splits; s += 32) {
       const long long base = ((long long)t * n_splits + s) * H + h;
       const float l = part_ml[base * 2 + 1];
-      if (l > 0.f) acc += __expf(part_ml[base * 2] - M) * part_o[base * r_kv + c];
+      const float w = (l > 0.f) ? __expf(part_ml[base * 2] - M) : 0.f;
+      if (s < 64) wsh[s] = w;
+      den += w * l;
     }
-    o_lat[((long long)t * H + h) * r_kv + c] = from_f32<T>(acc * inv);
+    den = warp_sum(den);
+    if (threadIdx.x == 0) inv_sh = den > 0.f ? 1.f / den : 0.f;
   }
+  __syncthreads();
+  const int c = threadIdx.x * 4;
+  if (c >= r_kv) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int ns = n_splits < 64 ? n_splits : 64;
+#pragma unroll 4
+  for (int s = 0; s < ns; ++s) {
+    const float w = wsh[s];
+    if (w == 0.f) continue;
+    const long long base = ((long long)t * n_splits + s) * H + h;
+    const float4 v = *reinterpret_cast<const float4*>(part_o + base * r_kv + c);
+    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  }
+  const float inv = inv_sh;
+  T* o = o_lat + ((long long)t * H + h) * r_kv + c;
+  o[0] = from_f32<T>(acc.x * inv); o[1] = from_f32<T>(acc.y * inv);
+  o[2] = from_f32<T>(acc.z * inv); o[3] = from_f32<T>(acc.w * inv);
 }
 
 // ---------------------------------------------------------------------------

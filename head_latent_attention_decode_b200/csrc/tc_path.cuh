@@ -146,15 +146,19 @@ static int launch_gemm_fp8(const CUtensorMap& A, const CUtensorMap& B, GemmArgs 
   }
 }
 
-// Splits of the K loop so that (M tiles x splits) fills the SMs about twice.
+// Splits of the K loop for a persistent grid of num_sms CTAs: minimise the
+// work of the busiest CTA, ceil(m_tiles * s / num_sms) units of 1/s of K each
+// (ties to fewer splits: fewer partial sums to add up afterwards).
 static int decode_splits_for(int m_tiles, int k_blocks, int num_sms) {
-  int s = (int)cdiv(2 * num_sms, m_tiles);
-  if (s > 16) s = 16;
-  if (s > k_blocks) s = k_blocks;
-  if (s < 1) s = 1;
-  // the launcher drops empty splits; report what it will use
-  const int per = (int)cdiv(k_blocks, s);
-  return (int)cdiv(k_blocks, per);
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 16 && s <= k_blocks; ++s) {
+    const int per = (int)cdiv(k_blocks, s);
+    const int real = (int)cdiv(k_blocks, per);          // the launcher drops empty splits
+    const double cost = (double)cdiv((long long)m_tiles * real, num_sms) * per;
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = real; }
+  }
+  return best;
 }
 
 // ---------------------------------------------------------------------------
@@ -174,14 +178,22 @@ struct FrontFoldTcArgs {
 //   q latent -> RMSNorm * q_norm_w -> qn (bf16)                          (r_q > 0)
 //   or q -> q_nope (bf16) and RoPE(q_pe) (bf16)                          (r_q = 0)
 //   kv latent -> RMSNorm * kv_norm_w, k_pe -> RoPE, row -> cache[slot]
-__global__ void __launch_bounds__(256) frontfold_tc_kernel(FrontFoldTcArgs p) {
+__global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
   extern __shared__ float y[];   // [N1]
   __shared__ float red[32];
   const int t = blockIdx.x;
+  const float* yp = p.Yp + (long long)t * p.N1;
   for (int c = threadIdx.x; c < p.N1; c += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < p.splits; ++s) acc += p.Yp[s * p.split_stride + (long long)t * p.N1 + c];
-    y[c] = acc;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;   // independent loads in flight
+    int s = 0;
+    for (; s + 4 <= p.splits; s += 4) {
+      a0 += yp[(s + 0) * p.split_stride + c];
+      a1 += yp[(s + 1) * p.split_stride + c];
+      a2 += yp[(s + 2) * p.split_stride + c];
+      a3 += yp[(s + 3) * p.split_stride + c];
+    }
+    for (; s < p.splits; ++s) a0 += yp[s * p.split_stride + c];
+    y[c] = (a0 + a1) + (a2 + a3);
   }
   __syncthreads();
   const int half = p.dr / 2;
@@ -401,7 +413,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   f.layout = c.row_layout; f.flag = flag;
   const size_t ff_smem = (size_t)L.N1 * 4;
   if (ff_smem > 48 * 1024) cudaFuncSetAttribute(frontfold_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ff_smem);
-  frontfold_tc_kernel<<<n, 256, ff_smem, s>>>(f);
+  frontfold_tc_kernel<<<n, 512, ff_smem, s>>>(f);
   mla_count_launch(1);
   // 3. q = qn @ wq_b with q_nope out and RoPE(q_pe) out (swap-AB)
   if (rq) {
