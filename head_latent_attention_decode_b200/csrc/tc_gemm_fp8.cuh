@@ -3,11 +3,13 @@
 // fp32 before the MAC with bf16 activations).
 //   D[b][m][n] = sum_kb scale[b][m/128][kb] * sum_{k in kb} e4m3(A[b][m][k]) * B[b][n][k]
 // A = the FP8 weight matrix (M = output features, 128 per tile = one scale row),
-// B = the bf16 tokens (N = BN). Per 128-wide K block:
-//   TMA brings the 128 x 128 code tile and the 2 x [BN x 64] bf16 token tiles;
-//   warps 0-3 decode the codes to bf16 (exact: every E4M3 value is a bf16
-//   value) into a 128-byte-swizzled tile;
-//   tcgen05 multiplies that block alone into one of two TMEM partials;
+// B = the tokens converted to f16 (N = BN; exact for |x| in f16's normal range,
+// which holds every activation of this layer). Per 128-wide K block:
+//   TMA brings the 128 x 128 code tile and the 2 x [BN x 64] f16 token tiles;
+//   warps 0-3 decode the codes to f16 with cvt.rn.f16x2.e4m3x2 (exact: every
+//   E4M3 value is an f16 value) into a 128-byte-swizzled tile;
+//   tcgen05 (kind::f16, f16 x f16 -> fp32) multiplies that block alone into one
+//   of two TMEM partials;
 //   warps 0-3 add scale * partial to fp32 registers.
 // So the scale multiplies each block's exact fp32 partial sum, the same value
 // as dequantising every weight in fp32 before the MAC, up to fp32 rounding.
@@ -30,20 +32,25 @@ struct Fp8Cfg {
   static constexpr int A8 = 128 * 128;             // FP8 code tile
   static constexpr int BB = BN * 64 * 2;           // one [BN x 64] bf16 tile
   static constexpr int STAGE = A8 + 2 * BB;
-  static constexpr int ABF = 2 * 128 * 64 * 2;     // decoded A: two [128 x 64] bf16 tiles
-  static constexpr int ST_RAW = (212 * 1024 - 2 * ABF - 512 - 1280) / STAGE;
+  static constexpr int ABF = 2 * 128 * 64 * 2;     // decoded A: two [128 x 64] f16 tiles
+  static constexpr int ST_RAW = (212 * 1024 - 2 * ABF - 1280) / STAGE;
   static constexpr int STAGES = ST_RAW > 6 ? 6 : ST_RAW;
   static constexpr int ABF_OFF = STAGES * STAGE;
-  static constexpr int LUT_OFF = ABF_OFF + 2 * ABF;
-  static constexpr int BAR_OFF = LUT_OFF + 512;
+  static constexpr int BAR_OFF = ABF_OFF + 2 * ABF;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;
   static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
 };
 
-// bf16 bits of an E4M3 code (from the OCP definition; every code is exact in bf16)
-__device__ __forceinline__ uint16_t e4m3_bf16_bits(uint32_t code) {
-  const float v = e4m3_to_f32((uint8_t)code);
-  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+// Two E4M3 codes (low byte -> low half) to two f16 values.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes16) {
+  uint32_t d;
+  const uint16_t a = (uint16_t)codes16;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(a));
+  return d;
+}
+// kind::f16 with f16 A and B, fp32 accumulator, K-major operands.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 template <int BN>
@@ -55,7 +62,6 @@ __global__ void __launch_bounds__(192, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  uint16_t* lut = (uint16_t*)(smem + C::LUT_OFF);
   const uint32_t bar = sbase + C::BAR_OFF;
   auto full_bar = [&](int s) { return bar + 8 * s; };
   auto empty_bar = [&](int s) { return bar + 8 * (C::STAGES + s); };
@@ -68,7 +74,6 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_word = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int c = threadIdx.x; c < 256; c += blockDim.x) lut[c] = e4m3_bf16_bits(c);
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int i = 0; i < 2; ++i) {
@@ -123,7 +128,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 5) {
     // ---------------- MMA issuer: one 128-wide K block into one TMEM partial ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, BN);
+      constexpr uint32_t idesc = idesc_f16(128, BN);
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
@@ -175,8 +180,8 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t outw[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          outw[2 * k] = (uint32_t)lut[w[k] & 0xFF] | ((uint32_t)lut[(w[k] >> 8) & 0xFF] << 16);
-          outw[2 * k + 1] = (uint32_t)lut[(w[k] >> 16) & 0xFF] | ((uint32_t)lut[w[k] >> 24] << 16);
+          outw[2 * k] = e4m3x2_to_f16x2(w[k] & 0xFFFF);
+          outw[2 * k + 1] = e4m3x2_to_f16x2(w[k] >> 16);
         }
         const int kk = q >> 2, c0 = 2 * (q & 3);
         uint8_t* orow = o0 + kk * 16384;

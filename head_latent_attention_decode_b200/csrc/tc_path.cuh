@@ -4,6 +4,7 @@
 // run in the GEMM epilogues or in one per-token front-fold kernel.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include "handle.cuh"
@@ -242,6 +243,22 @@ __global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
   }
 }
 
+// bf16 -> f16 copy (the FP8 GEMM's token operand), 8 elements per thread.
+__global__ void cvt_bf16_f16_kernel(const uint4* src, uint4* dst, long long n8) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+      const __half2 hh = __floats2half2_rn(f.x, f.y);
+      o[k] = *reinterpret_cast<const uint32_t*>(&hh);
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // out[n][m] = bf16(sum_s part[s][n][m])
 __global__ void splitk_reduce_bf16_kernel(const float* part, int splits, long long count, bf16* out) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
@@ -262,7 +279,7 @@ using namespace mla;
 using namespace mla::tc;
 
 struct TcDecodeWs {
-  size_t Yp, qn, q_nope, wo_part, total;
+  size_t Yp, qn, q_nope, wo_part, bf16c, total;
   int s1, s5;
 };
 
@@ -280,6 +297,14 @@ static TcDecodeWs tc_decode_ws(const mla_handle* h, long long n) {
   w.qn = put((size_t)n * (c.q_lora_rank ? c.q_lora_rank : 8) * 2);
   w.q_nope = put((size_t)n * c.n_heads * c.qk_nope * 2);
   w.wo_part = put((size_t)w.s5 * n * c.hidden * 4);
+  if (h->tc.fp8) {   // f16 copy of the largest token operand of an FP8 GEMM
+    long long e = c.hidden;
+    if (c.q_lora_rank > e) e = c.q_lora_rank;
+    if ((long long)c.n_heads * c.qk_nope > e) e = (long long)c.n_heads * c.qk_nope;
+    if ((long long)c.n_heads * c.kv_lora_rank > e) e = (long long)c.n_heads * c.kv_lora_rank;
+    if ((long long)c.n_heads * c.v_dim > e) e = (long long)c.n_heads * c.v_dim;
+    w.bf16c = put((size_t)n * e * 2 + 16);
+  }
   w.total = off;
   return w;
 }
@@ -346,16 +371,41 @@ static inline bool tc_decode_attn_supported(const mla_handle* h, int n, int) {
   return (h->tc.enabled && n <= 256) || (h->tc.fp8 && n <= 128);
 }
 
+static inline bool tc_attention_supported(const mla_handle* h) { return h->tc.attn != 0; }
+static inline bool tc_prefill_supported(const mla_handle* h, int) { return h->tc.enabled; }
+
 enum WSel { W_1, W_QB, W_UK, W_UV, W_O };
 
+// Token operand of a decode GEMM: a bf16 3-D view {K, d1, d2} (strides in
+// elements) over `elems` contiguous elements, rows in dimension rows_dim2 + 1.
+struct BView {
+  const void* p;
+  long long K, d1, d2, s1, s2, elems;
+  int rows_dim2;
+};
+
+static BView bview2(const void* p, long long K, long long rows) { return BView{p, K, rows, 1, K, K * rows, K * rows, 0}; }
+
 // Weight GEMM of the decode path: bf16 weights on tc_gemm_kernel, FP8 weights
-// on tc_gemm_fp8_kernel with the matrix's block scales.
-static int wgemm(const mla_handle* h, WSel w, const CUtensorMap& B, GemmArgs g, int bn, int splits, cudaStream_t s) {
+// on tc_gemm_fp8_kernel (tokens converted to f16 into `f16buf` first) with the
+// matrix's block scales.
+static int wgemm(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int bn, int splits, void* f16buf,
+                 cudaStream_t s) {
   const TcState& T = h->tc;
+  CUtensorMap B;
+  int st;
+  g.b_rows_dim2 = bv.rows_dim2;
   if (!T.fp8) {
+    if ((st = make_map(&B, bv.p, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
     const CUtensorMap* A = w == W_1 ? &T.a_W1 : w == W_QB ? &T.a_Wqb : w == W_UK ? &T.a_Wuk : w == W_UV ? &T.a_Wuv : &T.a_Wo;
     return launch_gemm(*A, B, g, bn, splits, T.num_sms, s);
   }
+  if ((((uintptr_t)bv.p) & 15) || (bv.elems % 8)) return MLA_ERR_UNSUPPORTED;
+  const long long n8 = bv.elems / 8;
+  const unsigned blocks = (unsigned)(cdiv(n8, 256) < 2048 ? cdiv(n8, 256) : 2048);
+  cvt_bf16_f16_kernel<<<blocks, 256, 0, s>>>((const uint4*)bv.p, (uint4*)f16buf, n8);
+  mla_count_launch(1);
+  if ((st = make_map(&B, f16buf, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
   const WeightLayout& L = h->L;
   const mla_config& c = h->cfg;
   const char* base = h->base;
@@ -373,8 +423,6 @@ static int wgemm(const mla_handle* h, WSel w, const CUtensorMap& B, GemmArgs g, 
   }
   return launch_gemm_fp8(*A, B, g, bn, splits, sc, ld, bs, T.num_sms, s);
 }
-static inline bool tc_attention_supported(const mla_handle* h) { return h->tc.attn != 0; }
-static inline bool tc_prefill_supported(const mla_handle* h, int) { return h->tc.enabled; }
 
 static GemmArgs gemm_args(int M, int N, int K, int batches, int mode, void* out, long long ldo, long long bstride,
                           int* flag) {
@@ -397,10 +445,9 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   const int bn = pick_bn(n);
   int st;
   // 1. Yp[split] = x @ W1 (swap-AB: A = W1 [N1, D], B = x [n, D])
-  CUtensorMap mx;
-  if ((st = make_map2(&mx, hidden, D, n, D, bn)) != MLA_OK) return st;
+  void* f16buf = tw + W.bf16c;
   GemmArgs g = gemm_args(L.N1, n, D, 1, EPI_F32_T, tw + W.Yp, L.N1, 0, flag);
-  if ((st = wgemm(h, W_1, mx, g, bn, W.s1, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_1, bview2(hidden, D, n), g, bn, W.s1, f16buf, s)) != MLA_OK) return st;
   // 2. split sum, norms, RoPE, scatter (and, without q_lora, q_nope / q_pe)
   FrontFoldTcArgs f{};
   f.Yp = (const float*)(tw + W.Yp); f.split_stride = (long long)n * L.N1; f.splits = W.s1; f.N1 = L.N1;
@@ -417,19 +464,16 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   mla_count_launch(1);
   // 3. q = qn @ wq_b with q_nope out and RoPE(q_pe) out (swap-AB)
   if (rq) {
-    CUtensorMap mq;
-    if ((st = make_map2(&mq, tw + W.qn, rq, n, rq, bn)) != MLA_OK) return st;
+
     GemmArgs g2 = gemm_args(L.Hq, n, rq, 1, EPI_QROPE_T, tw + W.q_nope, 0, 0, flag);
     g2.out2 = q_pe; g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr;
-    if ((st = wgemm(h, W_QB, mq, g2, bn, 1, s)) != MLA_OK) return st;
+    if ((st = wgemm(h, W_QB, bview2(tw + W.qn, rq, n), g2, bn, 1, f16buf, s)) != MLA_OK) return st;
   }
   // 4. q_abs[h] = q_nope[h] @ W_UK[h]  (batched over heads: A = Wuk[h] [r_kv, d_n], B = q_nope[:, h, :])
-  CUtensorMap mn;
-  if ((st = make_map(&mn, tw + W.q_nope, dn, H, n, (long long)dn * 2, (long long)H * dn * 2, bn, 1)) != MLA_OK)
-    return st;
+  const BView vn{tw + W.q_nope, dn, H, n, dn, (long long)H * dn, (long long)n * H * dn, 1};
   GemmArgs g3 = gemm_args(rkv, n, dn, H, EPI_BF16_T, q_abs, (long long)H * rkv, rkv, flag);
   g3.b_rows_dim2 = 1;
-  return wgemm(h, W_UK, mn, g3, bn, 1, s);
+  return wgemm(h, W_UK, vn, g3, bn, 1, f16buf, s);
 }
 
 // Split-KV absorbed attention and the LSE merge of the splits -> o_lat (bf16).
@@ -562,16 +606,14 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
                              part_ml, splits, o_lat, flag, s);
   if (st != MLA_OK) return st;
   // 2. head_out[h] = o_lat[h] @ W_UV[h]  (A = Wuv[h] [d_v, r_kv], B = o_lat[:, h, :])
-  CUtensorMap mo;
-  if ((st = make_map(&mo, o_lat, rkv, H, n, (long long)rkv * 2, (long long)H * rkv * 2, bn, 1)) != MLA_OK) return st;
+  void* f16buf = tw + W.bf16c;
+  const BView vo{o_lat, rkv, H, n, rkv, (long long)H * rkv, (long long)n * H * rkv, 1};
   GemmArgs g4 = gemm_args(dv, n, rkv, H, EPI_BF16_T, head, (long long)H * dv, dv, flag);
   g4.b_rows_dim2 = 1;
-  if ((st = wgemm(h, W_UV, mo, g4, bn, 1, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_UV, vo, g4, bn, 1, f16buf, s)) != MLA_OK) return st;
   // 3. out = head_out @ wo  (swap-AB, K split, then reduce to bf16)
-  CUtensorMap mh;
-  if ((st = make_map2(&mh, head, (long long)H * dv, n, (long long)H * dv, bn)) != MLA_OK) return st;
   GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
-  if ((st = wgemm(h, W_O, mh, g5, bn, W.s5, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n), g5, bn, W.s5, f16buf, s)) != MLA_OK) return st;
   const long long cnt = (long long)n * D;
   splitk_reduce_bf16_kernel<<<(unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s>>>(
       (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);
