@@ -92,7 +92,7 @@ def prefill_flops(s: wl.MlaShape, S: int) -> dict:
 
 KERNEL_SOURCES = {
     "tc_attn_decode_kernel": "tc_attn.cuh",
-    "tc_attn_small_kernel": "tc_attn_small.cuh",
+    "tc_attn_pair_kernel": "tc_attn_pair.cuh",
     "tc_prefill_attn_kernel": "tc_prefill_attn.cuh",
 }
 
@@ -100,7 +100,7 @@ KERNEL_SOURCES = {
 def dominant_kernel(w: wl.Workload) -> str:
     if w.mode == "prefill":
         return "tc_prefill_attn_kernel"
-    return "tc_attn_small_kernel" if w.shape.n_heads <= 32 else "tc_attn_decode_kernel"
+    return "tc_attn_pair_kernel" if w.shape.n_heads <= 32 else "tc_attn_decode_kernel"
 
 
 def measured_traffic(kernel: str, workload: str):

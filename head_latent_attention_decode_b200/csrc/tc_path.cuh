@@ -12,7 +12,7 @@
 #include "tc_gemm.cuh"
 #include "tc_gemm_fp8.cuh"
 #include "tc_attn.cuh"
-#include "tc_attn_small.cuh"
+#include "tc_attn_pair.cuh"
 #include "tc_prefill_attn.cuh"
 
 namespace mla {
@@ -59,6 +59,26 @@ static int make_map(CUtensorMap* m, const void* base, long long K, long long d1,
 // 2-D row-major [rows, K] bf16 matrix with row stride ld (elements).
 static int make_map2(CUtensorMap* m, const void* base, long long K, long long rows, long long ld, int box_rows) {
   return make_map(m, base, K, rows, 1, ld * 2, ld * 2 * rows, box_rows, 0);
+}
+
+// The paged cache [rows, R] bf16 (R a multiple of 64, rows a multiple of 8)
+// as a 4-D map {64 columns, 8 rows, R / 64 column groups, rows / 8 octets}, so
+// that one box brings `groups` adjacent 64-column k-blocks of 64 rows: in
+// shared memory [octet][group][8 rows][128 B], a 128-byte-swizzle operand
+// whose 8-row groups lie groups x 1024 B apart. Few large boxes stream faster
+// than many [64 x 64] ones.
+static int make_map_cache_groups(CUtensorMap* m, const void* base, long long R, long long rows, int groups) {
+  auto fn = encode_fn();
+  if (!fn) return MLA_ERR_CUDA;
+  if (((uintptr_t)base) & 15 || R % 64 || rows % 8) return MLA_ERR_UNSUPPORTED;
+  cuuint64_t dims[4] = {64, 8, (cuuint64_t)(R / 64), (cuuint64_t)(rows / 8)};
+  cuuint64_t strides[3] = {(cuuint64_t)(R * 2), 128, (cuuint64_t)(8 * R * 2)};
+  cuuint32_t box[4] = {64, 8, (cuuint32_t)groups, 8};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
 template <int BN>
@@ -491,26 +511,28 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
   const bool latent_ok = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && (((uintptr_t)q_abs) & 15) == 0 &&
                          (((uintptr_t)q_pe) & 15) == 0;
   if (latent_ok && H <= 32) {
-    // few heads: transposed tiles, one CTA per (sequence, split). Pick the
-    // split length (whole 128-row tiles) that minimises waves x tiles per CTA.
+    // few heads: transposed tiles, one 2-CTA cluster per (sequence, split).
+    // Pick the split length (whole 128-row tiles) that minimises waves x tiles
+    // per cluster.
     const int sms = T.num_sms > 0 ? T.num_sms : 148;
     const int tiles = (int)cdiv(max_ctx, 128);
     int best_ct = tiles, best_cost = 1 << 30;
     for (int ct = 1; ct <= tiles; ++ct) {
       const int spl = (int)cdiv(tiles, ct);
       if (spl > splits) continue;
-      const int waves = (int)cdiv((long long)n * spl, sms);
-      const int cost = waves * (ct + 2);   // + per-CTA set-up, in tiles
+      const int waves = (int)cdiv(2LL * n * spl, sms);
+      const int cost = waves * (ct + 2);   // + per-cluster set-up, in tiles
       if (cost < best_cost) { best_cost = cost; best_ct = ct; }
     }
     const int chunk = best_ct * 128;
     const int sp = (int)cdiv(max_ctx, chunk);
     splits = sp;
     const int NH = H <= 16 ? 16 : 32;
-    CUtensorMap mqa, mqp, mc;
+    CUtensorMap mqa, mqp, mc, ml;
     if ((st = make_map2(&mqa, q_abs, rkv, (long long)n * H, rkv, NH)) != MLA_OK) return st;
     if ((st = make_map2(&mqp, q_pe, dr, (long long)n * H, dr, NH)) != MLA_OK) return st;
     if ((st = make_map2(&mc, kv_cache, R, (long long)n_blocks * c.block_size, R, 64)) != MLA_OK) return st;
+    if ((st = make_map_cache_groups(&ml, kv_cache, R, (long long)n_blocks * c.block_size, 2)) != MLA_OK) return st;
     TcAttnArgs ta{};
     ta.n = n; ta.H = H; ta.splits = sp; ta.chunk = chunk;
     ta.bs = c.block_size; ta.n_blocks = n_blocks; ta.mbps = mbps; ta.max_ctx = max_ctx;
@@ -525,18 +547,18 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     mla_timer_begin("attn", s);
     if (NH == 16) {
       if (dev < 64 && !attr16[dev]) {
-        cudaFuncSetAttribute(tc_attn_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnSmallSmem<16>::SIZE);
+        cudaFuncSetAttribute(tc_attn_pair_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnPairSmem<16>::SIZE);
         attr16[dev] = true;
       }
-      tc_attn_small_kernel<16><<<n * sp, 192, AttnSmallSmem<16>::SIZE, s>>>(mqa, mqp, mc, ta);
+      tc_attn_pair_kernel<16><<<2 * n * sp, 224, AttnPairSmem<16>::SIZE, s>>>(mqa, mqp, mc, ml, ta);
     } else {
       if (dev < 64 && !attr32[dev]) {
-        cudaFuncSetAttribute(tc_attn_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnSmallSmem<32>::SIZE);
+        cudaFuncSetAttribute(tc_attn_pair_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnPairSmem<32>::SIZE);
         attr32[dev] = true;
       }
-      tc_attn_small_kernel<32><<<n * sp, 192, AttnSmallSmem<32>::SIZE, s>>>(mqa, mqp, mc, ta);
+      tc_attn_pair_kernel<32><<<2 * n * sp, 224, AttnPairSmem<32>::SIZE, s>>>(mqa, mqp, mc, ml, ta);
     }
     mla_timer_end("attn", s);
     mla_count_launch(1);

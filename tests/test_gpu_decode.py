@@ -60,6 +60,21 @@ def test_v2lite_bf16_small():
     check_case(case)
 
 
+def test_v2lite_bf16_ragged_single_tiles():
+    # contexts of 1 to 300 rows: units of one, two and three 128-row tiles, so
+    # the rotary block falls on either CTA of the pair and tails are ragged
+    case = DecodeCase(wl.WORKLOADS["v2lite_bf16"], batch=7, ctx=(1, 300)).run()
+    check_case(case)
+
+
+def test_v2lite_bf16_24_heads():
+    # 17..32 heads take the 32-column variant of the few-head attention kernel
+    w = dataclasses.replace(wl.WORKLOADS["v2lite_bf16"],
+                            shape=dataclasses.replace(wl.V2LITE, n_heads=24))
+    case = DecodeCase(w, batch=3, ctx=(200, 900)).run()
+    check_case(case)
+
+
 def test_v3_bf16_small_ragged():
     case = DecodeCase(wl.WORKLOADS["v3_bf16"], batch=5, ctx=(1, 2500)).run()
     check_case(case)
@@ -167,6 +182,20 @@ def test_bad_block_and_context_set_flags():
     torch.cuda.synchronize()
     assert case.flag() & mla.MLA_FLAG_BAD_CONTEXT
     mla.mla_clear_device_flag(case.layer.ws)
+
+
+def test_bad_block_on_tensor_core_path_sets_flag():
+    import head_latent_attention_decode_b200 as mla
+    for name in ("v2lite_bf16", "v3_bf16"):
+        case = DecodeCase(wl.WORKLOADS[name], batch=2, ctx=(150, 300)).run()
+        assert case.flag() == 0
+        table = case.table.clone()
+        table[1, 1] = case.cache.shape[0] + 7      # out of range block id: rows read as zeros, flag set
+        table[0, 0] = -3
+        case.layer.decode_attn(case.q_abs, case.q_pe, case.cache, table, case.ctx, case.max_ctx)
+        torch.cuda.synchronize()
+        assert case.flag() & mla.MLA_FLAG_BAD_BLOCK
+        mla.mla_clear_device_flag(case.layer.ws)
 
 
 def test_context_of_one():
