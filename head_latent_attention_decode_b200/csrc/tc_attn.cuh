@@ -75,7 +75,7 @@ __device__ __forceinline__ int attn_tile_rows(const TcAttnArgs& a, int b, int j0
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_qpe, const __grid_constant__ CUtensorMap tm_cache,
-                          TcAttnArgs a) {
+                          const __grid_constant__ CUtensorMap tm_lat, TcAttnArgs a) {
   using SM = AttnSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -145,6 +145,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       prefetch_tmap(&tm_cache);
+      prefetch_tmap(&tm_lat);
       if (r == 0) {
         mbar_arrive_expect_tx(qr_full, 16384);
         tma_load_3d(qr_s, &tm_qpe, qr_full, 0, b * a.H, 0);
@@ -157,8 +158,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         if (attn_tile_rows(a, b, r0 + 64 * t, r1, &row) < 0 && r == 0) set_flag(a.flag, MLA_FLAG_BAD_BLOCK);
         mbar_arrive_expect_tx(full_b + 8 * st, nkb * 8192);
         const uint32_t dst = tile_s + st * SM::STAGE;
-        for (int j = 0; j < 4; ++j)
-          tma_load_3d(dst + j * 8192, &tm_cache, full_b + 8 * st, a.lat_col0 + (int)r * 256 + 64 * j, (int)row, 0);
+        // the 4 latent k-blocks of the 64 rows in one box: [8 row octets][4 k-blocks][8 rows][128 B]
+        tma_load_4d(dst, &tm_lat, full_b + 8 * st, 0, 0, a.lat_col0 / 64 + 4 * (int)r, (int)(row / 8));
         if (r == 0) tma_load_3d(dst + 4 * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
         if (trace && t < 64) trace[t * 16 + 10] = global_timer_ns();
       }
@@ -181,6 +182,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       bool ok = mbar_wait(q_ready, 0, abort_word, a.flag);
       if (ok && r == 0) ok = mbar_wait(qr_full, 0, abort_word, a.flag);
       tc_fence_after();
+      // descriptors built once; stages and k-steps add their byte offset >> 4
+      const uint64_t d_t = sdesc_sw128_sbo(tile_s, 4096), d_rope = sdesc_sw128(tile_s + 4 * 8192);
+      const uint64_t d_qr = sdesc_sw128(qr_s), d_v = sdesc_sw128_mn_sbo(tile_s, 1024, 4096);
       int next_s = 0, next_o = 0;
       uint64_t t_last = global_timer_ns();
       while (ok && next_o < T) {
@@ -189,18 +193,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
           const int t = next_s, st = t % ATT_NST, sb = t & 1;
           if (mbar_test(full_b + 8 * st, (t / ATT_NST) & 1) && mbar_test(sp_empty_b + 8 * sb, ((t >> 1) & 1) ^ 1)) {
             tc_fence_after();
-            const uint32_t tl = tile_s + st * SM::STAGE;
+            const uint64_t dt = d_t + (uint64_t)(st * (SM::STAGE / 16));
             const uint32_t d = tmem + ATT_TM_S + 64 * sb;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
               for (int k = 0; k < 4; ++k)
-                mma_bf16_ts(d, tmem + ATT_TM_Q + 32 * j + 8 * k, sdesc_sw128(tl + j * 8192 + 32 * k), idesc_s,
+                mma_bf16_ts(d, tmem + ATT_TM_Q + 32 * j + 8 * k, dt + (j * 1024 + 32 * k) / 16, idesc_s,
                             (j > 0 || k > 0) ? 1u : 0u);
             if (r == 0) {
+              const uint64_t dr = d_rope + (uint64_t)(st * (SM::STAGE / 16));
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16(d, sdesc_sw128(qr_s + 32 * k), sdesc_sw128(tl + 4 * 8192 + 32 * k), idesc_s, 1u);
+              for (int k = 0; k < 4; ++k) mma_bf16(d, d_qr + 2 * k, dr + 2 * k, idesc_s, 1u);
             }
             mma_commit(s_full_b + 8 * sb);
             if (trace && t < 64) trace[t * 16 + 8] = global_timer_ns();
@@ -212,11 +216,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
           const int u = next_o, st = u % ATT_NST, sb = u & 1;
           if (mbar_test(p_full_b + 8 * sb, (u >> 1) & 1)) {
             tc_fence_after();
-            const uint32_t v = tile_s + st * SM::STAGE;
+            const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              mma_bf16_ts(tmem + ATT_TM_O, tmem + ATT_TM_S + 64 * sb + 8 * k, sdesc_sw128_mn(v + 2048 * k, 8192),
-                          idesc_o, (u > 0 || k > 0) ? 1u : 0u);
+              mma_bf16_ts(tmem + ATT_TM_O, tmem + ATT_TM_S + 64 * sb + 8 * k, dv + 8192 * k / 16, idesc_o,
+                          (u > 0 || k > 0) ? 1u : 0u);
             mma_commit(o_done);
             mma_commit(sp_empty_b + 8 * sb);
             mma_commit(empty_b + 8 * st);
@@ -233,6 +237,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
           *abort_word = 1;
           set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT);
           ok = false;
+        } else {
+          __nanosleep(32);   // leave the issue slots to the softmax warp on this sub-partition
         }
       }
       mma_commit(fin);
@@ -378,11 +384,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       if (valid < 64) {
         // rows past the context may hold anything (even NaN); P is 0 there, but
         // 0 * NaN is not, so clear them in the four latent slots before P.V
+        // latent rows are laid out [8 row octets][4 k-blocks][8 rows][128 B]
         uint8_t* tl = smem + SM::TILE_OFF + st * SM::STAGE;
-        const int nbytes = (64 - valid) * 128;
-        for (int i = h * 16; i < 4 * nbytes; i += 128 * 16) {
-          const int j = i / nbytes, off = i % nbytes;
-          *reinterpret_cast<uint4*>(tl + j * 8192 + valid * 128 + off) = make_uint4(0, 0, 0, 0);
+        for (int row = valid + (h >> 1); row < 64; row += 64) {
+          uint8_t* rp = tl + (row >> 3) * 4096 + (row & 7) * 128 + (h & 1) * 2048;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)   // two of the four k-blocks: 256 bytes
+            *reinterpret_cast<uint4*>(rp + (c >> 3) * 1024 + 16 * (c & 7)) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }

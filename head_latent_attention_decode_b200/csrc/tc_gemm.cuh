@@ -249,6 +249,8 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, BN);
+      // descriptors built once; stages and k-steps add their byte offset >> 4
+      const uint64_t da0 = sdesc_sw128(a_base), db0 = sdesc_sw128(b_base);
       int it = 0, tile = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x, ++tile) {
@@ -263,10 +265,9 @@ __global__ void __launch_bounds__(192, 1)
           const int st = it % C::STAGES, round = it / C::STAGES;
           if (!mbar_wait(full_bar(st), round & 1, abort_word, g.flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = a_base + st * C::A_BYTES, sb = b_base + st * C::B_BYTES;
+          const uint64_t da = da0 + (uint64_t)(st * (C::A_BYTES / 16)), db = db0 + (uint64_t)(st * (C::B_BYTES / 16));
 #pragma unroll
-          for (int k = 0; k < C::BK / 16; ++k)
-            mma_bf16(d, sdesc_sw128(sa + 32 * k), sdesc_sw128(sb + 32 * k), idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < C::BK / 16; ++k) mma_bf16(d, da + 2 * k, db + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           mma_commit(empty_bar(st));
         }
         if (!ok) break;

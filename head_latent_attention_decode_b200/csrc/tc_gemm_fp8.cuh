@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------- MMA issuer: one 128-wide K block into one TMEM partial ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, BN);
+      // descriptors built once; buffers and k-steps add their byte offset >> 4
+      const uint64_t da0 = sdesc_sw128(sbase + C::ABF_OFF), db0 = sdesc_sw128(sbase + C::A8);
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
@@ -141,14 +143,13 @@ __global__ void __launch_bounds__(192, 1)
           if (!mbar_wait(conv_full + 8 * cb, (it >> 1) & 1, abort_word, g.flag)) { ok = false; break; }
           if (!mbar_wait(part_free + 8 * cb, ((it >> 1) & 1) ^ 1, abort_word, g.flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a = sbase + C::ABF_OFF + cb * C::ABF;
-          const uint32_t bt = sbase + st * C::STAGE + C::A8;
+          const uint64_t da = da0 + (uint64_t)(cb * (C::ABF / 16)), db = db0 + (uint64_t)(st * (C::STAGE / 16));
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              mma_bf16(tmem + cb * BN, sdesc_sw128(a + kk * 16384 + 32 * k), sdesc_sw128(bt + kk * C::BB + 32 * k),
-                       idesc, (kk > 0 || k > 0) ? 1u : 0u);
+              mma_bf16(tmem + cb * BN, da + (kk * 16384 + 32 * k) / 16, db + (kk * C::BB + 32 * k) / 16, idesc,
+                       (kk > 0 || k > 0) ? 1u : 0u);
           mma_commit(part_full + 8 * cb);
           mma_commit(conv_free + 8 * cb);
           mma_commit(empty_bar(st));

@@ -204,17 +204,29 @@ __global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* yp = p.Yp + (long long)t * p.N1;
-  for (int c = threadIdx.x; c < p.N1; c += blockDim.x) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;   // independent loads in flight
-    int s = 0;
-    for (; s + 4 <= p.splits; s += 4) {
-      a0 += yp[(s + 0) * p.split_stride + c];
-      a1 += yp[(s + 1) * p.split_stride + c];
-      a2 += yp[(s + 2) * p.split_stride + c];
-      a3 += yp[(s + 3) * p.split_stride + c];
+  if (p.N1 % 4 == 0 && p.split_stride % 4 == 0 && ((uintptr_t)p.Yp & 15) == 0) {
+    // 16-byte loads, the first eight splits' loads all in flight before the sum
+    const float4* yp4 = reinterpret_cast<const float4*>(yp);
+    const long long st4 = p.split_stride >> 2;
+    for (int c = threadIdx.x; c < (p.N1 >> 2); c += blockDim.x) {
+      float4 v[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) v[s] = s < p.splits ? yp4[s * st4 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 acc = v[0];
+#pragma unroll
+      for (int s = 1; s < 8; ++s) { acc.x += v[s].x; acc.y += v[s].y; acc.z += v[s].z; acc.w += v[s].w; }
+      for (int s = 8; s < p.splits; ++s) {
+        const float4 w = yp4[s * st4 + c];
+        acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
+      }
+      reinterpret_cast<float4*>(y)[c] = acc;
     }
-    for (; s < p.splits; ++s) a0 += yp[s * p.split_stride + c];
-    y[c] = (a0 + a1) + (a2 + a3);
+  } else {
+    for (int c = threadIdx.x; c < p.N1; c += blockDim.x) {
+      float acc = 0.f;
+      for (int s = 0; s < p.splits; ++s) acc += yp[s * p.split_stride + c];
+      y[c] = acc;
+    }
   }
   __syncthreads();
   const int half = p.dr / 2;
@@ -572,9 +584,10 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     const int chunk = (int)cdiv(cdiv(max_ctx, sp), 64) * 64;
     sp = (int)cdiv(max_ctx, chunk);
     splits = sp;
-    CUtensorMap mqp, mc;
+    CUtensorMap mqp, mc, ml;
     if ((st = make_map2(&mqp, q_pe, dr, (long long)n * H, dr, 128)) != MLA_OK) return st;
     if ((st = make_map2(&mc, kv_cache, R, (long long)n_blocks * c.block_size, R, 64)) != MLA_OK) return st;
+    if ((st = make_map_cache_groups(&ml, kv_cache, R, (long long)n_blocks * c.block_size, 4)) != MLA_OK) return st;
     TcAttnArgs ta{};
     ta.n = n; ta.H = H; ta.splits = sp; ta.chunk = chunk;
     ta.bs = c.block_size; ta.n_blocks = n_blocks; ta.mbps = mbps; ta.max_ctx = max_ctx;
@@ -591,7 +604,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
       attr[dev] = true;
     }
     mla_timer_begin("attn", s);
-    tc_attn_decode_kernel<<<2 * n * sp, 320, AttnSmem::SIZE, s>>>(mqp, mc, ta);
+    tc_attn_decode_kernel<<<2 * n * sp, 320, AttnSmem::SIZE, s>>>(mqp, mc, ml, ta);
     mla_timer_end("attn", s);
     mla_count_launch(1);
   } else {

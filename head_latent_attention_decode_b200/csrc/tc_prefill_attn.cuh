@@ -110,6 +110,9 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc_s = idesc_bf16(128, 128);
       constexpr uint32_t idesc_o = idesc_bf16(128, 128, 1);
       bool ok = mbar_wait(q_full, 0, abort_word, a.flag);
+      // descriptors built once; buffers and k-steps add their byte offset >> 4
+      const uint64_t d_q = sdesc_sw128(q_s), d_k = sdesc_sw128(st_s);
+      const uint64_t d_v = sdesc_sw128_mn(st_s + 3 * 16384, 16384);
       int next_s = 0, next_o = 0;
       uint64_t t_last = global_timer_ns();
       while (ok && next_o < T) {
@@ -118,13 +121,13 @@ __global__ void __launch_bounds__(192, 1)
           const int t = next_s, st = t & 1;
           if (mbar_test(full_b + 8 * st, (t >> 1) & 1) && mbar_test(sp_empty_b + 8 * st, ((t >> 1) & 1) ^ 1)) {
             tc_fence_after();
-            const uint32_t kt = st_s + st * SM::STAGE;
+            const uint64_t dk = d_k + (uint64_t)(st * (SM::STAGE / 16));
 #pragma unroll
             for (int j = 0; j < 3; ++j)
 #pragma unroll
               for (int k = 0; k < 4; ++k)
-                mma_bf16(tmem + PA_TM_S + 128 * st, sdesc_sw128(q_s + j * 16384 + 32 * k),
-                         sdesc_sw128(kt + j * 16384 + 32 * k), idesc_s, (j > 0 || k > 0) ? 1u : 0u);
+                mma_bf16(tmem + PA_TM_S + 128 * st, d_q + (j * 16384 + 32 * k) / 16, dk + (j * 16384 + 32 * k) / 16,
+                         idesc_s, (j > 0 || k > 0) ? 1u : 0u);
             mma_commit(s_full_b + 8 * st);
             ++next_s;
             did = true;
@@ -134,11 +137,11 @@ __global__ void __launch_bounds__(192, 1)
           const int u = next_o, st = u & 1;
           if (mbar_test(p_full_b + 8 * st, (u >> 1) & 1)) {
             tc_fence_after();
-            const uint32_t v = st_s + st * SM::STAGE + 3 * 16384;
+            const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              mma_bf16_ts(tmem + PA_TM_O, tmem + PA_TM_S + 128 * st + 8 * k, sdesc_sw128_mn(v + 2048 * k, 16384),
-                          idesc_o, (u > 0 || k > 0) ? 1u : 0u);
+              mma_bf16_ts(tmem + PA_TM_O, tmem + PA_TM_S + 128 * st + 8 * k, dv + 2048 * k / 16, idesc_o,
+                          (u > 0 || k > 0) ? 1u : 0u);
             mma_commit(o_done);
             mma_commit(sp_empty_b + 8 * st);
             mma_commit(empty_b + 8 * st);
