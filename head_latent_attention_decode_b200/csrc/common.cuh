@@ -67,4 +67,14 @@ __device__ __forceinline__ void set_flag(int* flag, int bits) {
   if (flag) atomicOr(flag, bits);
 }
 
+// Programmatic dependent launch. griddep_wait: block until the grids this one
+// depends on have completed and their memory is visible (returns at once
+// without such a dependency). griddep_launch_dependents: let the next grid of
+// the stream launch once every CTA of this one has called it or exited; call it
+// only after this CTA holds its tensor memory, so that an early CTA of the next
+// grid can never take tensor memory that a CTA of this grid still waits for.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 }  // namespace mla

@@ -124,6 +124,8 @@ struct FrontFoldArgs {
 
 template <typename TACT>
 __global__ void __launch_bounds__(256) frontfold_epilogue_kernel(FrontFoldArgs p) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* y = p.Y + (long long)t * p.ldy;
@@ -303,6 +305,8 @@ __global__ void __launch_bounds__(256) attn_decode_simt_kernel(AttnArgs p) {
 template <typename T>
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, const float* part_ml, int n_splits,
                                                            int H, int r_kv, T* o_lat) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ float wsh[64];
   __shared__ float inv_sh;
   const int t = blockIdx.x, h = blockIdx.y;

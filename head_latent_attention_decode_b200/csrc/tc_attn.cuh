@@ -77,6 +77,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_qpe, const __grid_constant__ CUtensorMap tm_cache,
                           const __grid_constant__ CUtensorMap tm_lat, TcAttnArgs a) {
   using SM = AttnSmem;
+  griddep_wait();   // the inputs all come from the stream's earlier kernels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -140,6 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   cluster_sync_all();   // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 4) {
     // ---------------- TMA producer ----------------

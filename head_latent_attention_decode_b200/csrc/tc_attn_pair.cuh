@@ -49,6 +49,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
                         const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_lat,
                         TcAttnArgs a) {
   using SM = AttnPairSmem<NH>;
+  griddep_wait();   // the inputs all come from the stream's earlier kernels
   constexpr int NPR = SM::NPR, QKB = SM::QKB;
   constexpr int CPR = NH / 4;                  // 16-byte chunks per row of a partial
   constexpr int XSH = NH == 16 ? 1 : 0;        // chunk swizzle: 8 consecutive rows cover all 32 banks
@@ -134,6 +135,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
   cluster_sync_all();   // both CTAs' barriers exist before any remote arrive or st.async
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const uint32_t tm_s = tmem, tm_o = tmem + 2 * NH;   // S^T buffers [0,NH) [NH,2NH); O^T group g at 2NH + g NH
 
   if (warp == 4) {

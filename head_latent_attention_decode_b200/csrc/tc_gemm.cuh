@@ -40,6 +40,10 @@ struct GemmArgs {
   const float* sin;
   int H, dn, dr;
   int* flag;
+  // operand read from memory no earlier kernel of the stream writes (the
+  // weights): 1 = A, 2 = B, 0 = neither. Its first pipeline stages are loaded
+  // before waiting for the previous kernel.
+  int static_op;
 };
 
 template <int BN>
@@ -215,10 +219,37 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 4) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
+      auto load_a = [&](int st, int kb, int mt, int b) {
+        const int ar = mt * C::BM;
+        if (g.a_rows_dim2) tma_load_3d(a_base + st * C::A_BYTES, &tmA, full_bar(st), kb * C::BK, b, ar);
+        else tma_load_3d(a_base + st * C::A_BYTES, &tmA, full_bar(st), kb * C::BK, ar, b);
+      };
+      auto load_b = [&](int st, int kb, int nt, int b) {
+        const int br = nt * BN;
+        if (g.b_rows_dim2) tma_load_3d(b_base + st * C::B_BYTES, &tmB, full_bar(st), kb * C::BK, b, br);
+        else tma_load_3d(b_base + st * C::B_BYTES, &tmB, full_bar(st), kb * C::BK, br, b);
+      };
+      // the static operand of the first STAGES k-blocks goes out before the wait
+      const int npre = g.static_op ? C::STAGES : 0;
+      {
+        int it = 0;
+        for (int u = blockIdx.x; u < g.total_units && it < npre; u += gridDim.x) {
+          int mt, nt, b, s;
+          decode_unit(g, u, mt, nt, b, s);
+          const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
+          for (int kb = kb0; kb < kb1 && it < npre; ++kb, ++it) {
+            mbar_arrive_expect_tx(full_bar(it), C::STAGE_BYTES);
+            if (g.static_op == 1) load_a(it, kb, mt, b);
+            else load_b(it, kb, nt, b);
+          }
+        }
+      }
+      griddep_wait();
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
@@ -227,13 +258,15 @@ __global__ void __launch_bounds__(192, 1)
         const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int st = it % C::STAGES, round = it / C::STAGES;
+          if (it < npre) {   // the stage is armed and its static operand is on its way
+            if (g.static_op == 1) load_b(st, kb, nt, b);
+            else load_a(st, kb, mt, b);
+            continue;
+          }
           if (!mbar_wait(empty_bar(st), (round & 1) ^ 1, abort_word, g.flag)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(st), C::STAGE_BYTES);
-          const int ar = mt * C::BM, br = nt * BN;
-          if (g.a_rows_dim2) tma_load_3d(a_base + st * C::A_BYTES, &tmA, full_bar(st), kb * C::BK, b, ar);
-          else tma_load_3d(a_base + st * C::A_BYTES, &tmA, full_bar(st), kb * C::BK, ar, b);
-          if (g.b_rows_dim2) tma_load_3d(b_base + st * C::B_BYTES, &tmB, full_bar(st), kb * C::BK, b, br);
-          else tma_load_3d(b_base + st * C::B_BYTES, &tmB, full_bar(st), kb * C::BK, br, b);
+          load_a(st, kb, mt, b);
+          load_b(st, kb, nt, b);
         }
       }
       // drain: every load issued has landed before the CTA can exit
@@ -282,6 +315,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ---------------- epilogue: warps 0..3 <-> TMEM lanes 32w..32w+31 ----------------
+    griddep_wait();   // the output and the RoPE tables belong to the stream's earlier kernels
     int tile = 0;
     for (int u = blockIdx.x; u < g.total_units; u += gridDim.x, ++tile) {
       int mt, nt, b, s;

@@ -92,10 +92,26 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 4) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
+      // the weight codes of the first STAGES k-blocks go out before the wait for
+      // the previous kernel (no earlier kernel of the stream writes them)
+      {
+        int it = 0;
+        for (int u = blockIdx.x; u < g.total_units && it < C::STAGES; u += gridDim.x) {
+          int mt, nt, b, s;
+          decode_unit(g, u, mt, nt, b, s);
+          const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
+          for (int kb = kb0; kb < kb1 && it < C::STAGES; ++kb, ++it) {
+            mbar_arrive_expect_tx(full_bar(it), C::STAGE);
+            tma_load_3d(sbase + it * C::STAGE, &tmA, full_bar(it), kb * 128, mt * 128, b);
+          }
+        }
+      }
+      griddep_wait();
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
@@ -104,10 +120,12 @@ __global__ void __launch_bounds__(192, 1)
         const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int st = it % C::STAGES;
-          if (!mbar_wait(empty_bar(st), ((it / C::STAGES) & 1) ^ 1, abort_word, g.flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(st), C::STAGE);
           const uint32_t dst = sbase + st * C::STAGE;
-          tma_load_3d(dst, &tmA, full_bar(st), kb * 128, mt * 128, b);
+          if (it >= C::STAGES) {
+            if (!mbar_wait(empty_bar(st), ((it / C::STAGES) & 1) ^ 1, abort_word, g.flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(full_bar(st), C::STAGE);
+            tma_load_3d(dst, &tmA, full_bar(st), kb * 128, mt * 128, b);
+          }
           const int br = nt * BN;
           if (g.b_rows_dim2) {
             tma_load_3d(dst + C::A8, &tmB, full_bar(st), kb * 128, b, br);
@@ -162,6 +180,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ---------------- warps 0-3: decode codes, fold scaled partials, epilogue ----------------
+    griddep_wait();   // the output belongs to the stream's earlier kernels
     const int r = threadIdx.x;                 // A row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     float acc[BN];

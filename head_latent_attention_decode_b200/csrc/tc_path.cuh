@@ -81,6 +81,25 @@ static int make_map_cache_groups(CUtensorMap* m, const void* base, long long R, 
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel's CTAs may start
+// while the previous kernel of the stream drains (its launch latency and
+// set-up overlap that kernel); each kernel of this library calls griddep_wait
+// before it touches memory an earlier kernel writes.
+template <typename... KArgs, typename... Args>
+static void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 template <int BN>
 static int launch_gemm_bn(const CUtensorMap& A, const CUtensorMap& B, const GemmArgs& g, int num_sms,
                           cudaStream_t s) {
@@ -93,7 +112,7 @@ static int launch_gemm_bn(const CUtensorMap& A, const CUtensorMap& B, const Gemm
     attr_set[dev] = true;
   }
   const int grid = g.total_units < num_sms ? g.total_units : num_sms;
-  tc_gemm_kernel<BN><<<grid, 192, C::SMEM, s>>>(A, B, g);
+  launch_pdl(tc_gemm_kernel<BN>, grid, 192, C::SMEM, s, A, B, g);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -139,7 +158,7 @@ static int launch_gemm_fp8_bn(const CUtensorMap& A, const CUtensorMap& B, const 
     attr_set[dev] = true;
   }
   const int grid = fa.g.total_units < num_sms ? fa.g.total_units : num_sms;
-  tc_gemm_fp8_kernel<BN><<<grid, 192, C::SMEM, s>>>(A, B, fa);
+  launch_pdl(tc_gemm_fp8_kernel<BN>, grid, 192, C::SMEM, s, A, B, fa);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -200,6 +219,8 @@ struct FrontFoldTcArgs {
 //   or q -> q_nope (bf16) and RoPE(q_pe) (bf16)                          (r_q = 0)
 //   kv latent -> RMSNorm * kv_norm_w, k_pe -> RoPE, row -> cache[slot]
 __global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float y[];   // [N1]
   __shared__ float red[32];
   const int t = blockIdx.x;
@@ -277,6 +298,8 @@ __global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
 
 // bf16 -> f16 copy (the FP8 GEMM's token operand), 8 elements per thread.
 __global__ void cvt_bf16_f16_kernel(const uint4* src, uint4* dst, long long n8) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
     const uint4 v = src[i];
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -293,6 +316,8 @@ __global__ void cvt_bf16_f16_kernel(const uint4* src, uint4* dst, long long n8) 
 
 // out[n][m] = bf16(sum_s part[s][n][m])
 __global__ void splitk_reduce_bf16_kernel(const float* part, int splits, long long count, bf16* out) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
        i += (long long)gridDim.x * blockDim.x) {
     float acc = 0.f;
@@ -435,7 +460,7 @@ static int wgemm(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int b
   if ((((uintptr_t)bv.p) & 15) || (bv.elems % 8)) return MLA_ERR_UNSUPPORTED;
   const long long n8 = bv.elems / 8;
   const unsigned blocks = (unsigned)(cdiv(n8, 256) < 2048 ? cdiv(n8, 256) : 2048);
-  cvt_bf16_f16_kernel<<<blocks, 256, 0, s>>>((const uint4*)bv.p, (uint4*)f16buf, n8);
+  launch_pdl(cvt_bf16_f16_kernel, blocks, 256, 0, s, (const uint4*)bv.p, (uint4*)f16buf, n8);
   mla_count_launch(1);
   if ((st = make_map(&B, f16buf, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
   const WeightLayout& L = h->L;
@@ -461,6 +486,8 @@ static GemmArgs gemm_args(int M, int N, int K, int batches, int mode, void* out,
   GemmArgs g{};
   g.M = M; g.N = N; g.K = K; g.batches = batches; g.mode = mode; g.out = out; g.ldo = ldo; g.bstride = bstride;
   g.flag = flag;
+  // decode GEMMs run swap-AB (A = the weights), prefill GEMMs with B = the weights
+  g.static_op = (mode == EPI_F32_T || mode == EPI_BF16_T || mode == EPI_QROPE_T) ? 1 : 2;
   return g;
 }
 
@@ -492,7 +519,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   f.layout = c.row_layout; f.flag = flag;
   const size_t ff_smem = (size_t)L.N1 * 4;
   if (ff_smem > 48 * 1024) cudaFuncSetAttribute(frontfold_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ff_smem);
-  frontfold_tc_kernel<<<n, 512, ff_smem, s>>>(f);
+  launch_pdl(frontfold_tc_kernel, n, 512, ff_smem, s, f);
   mla_count_launch(1);
   // 3. q = qn @ wq_b with q_nope out and RoPE(q_pe) out (swap-AB)
   if (rq) {
@@ -563,14 +590,14 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
                              AttnPairSmem<16>::SIZE);
         attr16[dev] = true;
       }
-      tc_attn_pair_kernel<16><<<2 * n * sp, 224, AttnPairSmem<16>::SIZE, s>>>(mqa, mqp, mc, ml, ta);
+      launch_pdl(tc_attn_pair_kernel<16>, 2 * n * sp, 224, AttnPairSmem<16>::SIZE, s, mqa, mqp, mc, ml, ta);
     } else {
       if (dev < 64 && !attr32[dev]) {
         cudaFuncSetAttribute(tc_attn_pair_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnPairSmem<32>::SIZE);
         attr32[dev] = true;
       }
-      tc_attn_pair_kernel<32><<<2 * n * sp, 224, AttnPairSmem<32>::SIZE, s>>>(mqa, mqp, mc, ml, ta);
+      launch_pdl(tc_attn_pair_kernel<32>, 2 * n * sp, 224, AttnPairSmem<32>::SIZE, s, mqa, mqp, mc, ml, ta);
     }
     mla_timer_end("attn", s);
     mla_count_launch(1);
@@ -604,7 +631,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
       attr[dev] = true;
     }
     mla_timer_begin("attn", s);
-    tc_attn_decode_kernel<<<2 * n * sp, 320, AttnSmem::SIZE, s>>>(mqp, mc, ml, ta);
+    launch_pdl(tc_attn_decode_kernel, 2 * n * sp, 320, AttnSmem::SIZE, s, mqp, mc, ml, ta);
     mla_timer_end("attn", s);
     mla_count_launch(1);
   } else {
@@ -621,7 +648,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     mla_timer_end("attn", s);
     mla_count_launch(1);
   }
-  attn_combine_kernel<bf16><<<dim3(n, H), 128, 0, s>>>(part_o, part_ml, splits, H, rkv, o_lat);
+  launch_pdl(attn_combine_kernel<bf16>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits, H, rkv, o_lat);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -650,8 +677,8 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
   if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n), g5, bn, W.s5, f16buf, s)) != MLA_OK) return st;
   const long long cnt = (long long)n * D;
-  splitk_reduce_bf16_kernel<<<(unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s>>>(
-      (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);
+  launch_pdl(splitk_reduce_bf16_kernel, (unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s,
+             (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -692,7 +719,7 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
   f.cache = kv_cache; f.n_rows = (long long)n_blocks * c.block_size;
   f.slot = slot_mapping; f.layout = c.row_layout; f.flag = flag;
   f.cn = ws + pcn; f.kpe = ws + pkpe;
-  frontfold_epilogue_kernel<bf16><<<S, 256, 0, s>>>(f);
+  launch_pdl(frontfold_epilogue_kernel<bf16>, S, 256, 0, s, f);
   mla_count_launch(1);
   if (rq) {
     CUtensorMap mq;
@@ -723,7 +750,7 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
       attr[dev] = true;
     }
     mla_timer_begin("prefill_attn", s);
-    tc_prefill_attn_kernel<<<pa.q_tiles * H, 192, PaSmem::SIZE, s>>>(mq, mkv, mkpe, pa);
+    launch_pdl(tc_prefill_attn_kernel, pa.q_tiles * H, 192, PaSmem::SIZE, s, mq, mkv, mkpe, pa);
     mla_timer_end("prefill_attn", s);
     mla_count_launch(1);
   } else {

@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                            const __grid_constant__ CUtensorMap tm_kpe, TcPrefillAttnArgs a) {
   using SM = PaSmem;
+  griddep_wait();   // the inputs all come from the stream's earlier kernels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 4) {
     // ---------------- TMA producer ----------------
