@@ -6,11 +6,11 @@
 // B = the tokens converted to f16 (N = BN; exact for |x| in f16's normal range,
 // which holds every activation of this layer). Per 128-wide K block:
 //   TMA brings the 128 x 128 code tile and the 2 x [BN x 64] f16 token tiles;
-//   warps 0-3 decode the codes to f16 with cvt.rn.f16x2.e4m3x2 (exact: every
+//   warps 0-7 decode the codes to f16 with cvt.rn.f16x2.e4m3x2 (exact: every
 //   E4M3 value is an f16 value) into a 128-byte-swizzled tile;
 //   tcgen05 (kind::f16, f16 x f16 -> fp32) multiplies that block alone into one
 //   of two TMEM partials;
-//   warps 0-3 add scale * partial to fp32 registers.
+//   warps 0-7 add scale * partial to fp32 registers (two column halves).
 // So the scale multiplies each block's exact fp32 partial sum, the same value
 // as dequantising every weight in fp32 before the MAC, up to fp32 rounding.
 // The epilogue modes are those of tc_gemm.cuh.
@@ -53,8 +53,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// warps 0-7 decode the codes (warpgroup h: k-half h of every row) and fold the
+// scaled partials (warpgroup h: column half h, or all columns by warps 0-3 when
+// BN < 32); warp 8 issues TMA, warp 9 the MMAs.
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     tc_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        Fp8GemmArgs fa) {
   using C = Fp8Cfg<BN>;
@@ -77,16 +80,16 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(conv_full + 8 * i, 128);
+      mbar_init(conv_full + 8 * i, 256);
       mbar_init(conv_free + 8 * i, 1);
       mbar_init(part_full + 8 * i, 1);
-      mbar_init(part_free + 8 * i, 128);
+      mbar_init(part_free + 8 * i, BN >= 32 ? 256 : 128);
     }
     mbar_init(fin, 1);
     *abort_word = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
+  if (warp == 8 && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
   if (warp == 0) { tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       // the weight codes of the first STAGES k-blocks go out before the wait for
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(192, 1)
           if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(g.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer: one 128-wide K block into one TMEM partial ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, BN);
@@ -179,22 +182,29 @@ __global__ void __launch_bounds__(192, 1)
         if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(g.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
     }
   } else {
-    // ---------------- warps 0-3: decode codes, fold scaled partials, epilogue ----------------
+    // ---------------- warps 0-7: decode codes, fold scaled partials, epilogue ----------------
     griddep_wait();   // the output belongs to the stream's earlier kernels
-    const int r = threadIdx.x;                 // A row of the tile = TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float acc[BN];
+    constexpr int FSPLIT = BN >= 32 ? 2 : 1;   // warpgroups that fold
+    constexpr int NCOL = BN / FSPLIT;          // columns each folding thread owns
+    const int t = threadIdx.x;
+    const int r = t & 127;                     // A row of the tile = TMEM lane
+    const int half = t >> 7;                   // warpgroup: k-half to decode, column half to fold
+    const bool folds = half < FSPLIT;
+    const int col0 = half * NCOL;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    float acc[NCOL];
     int it = 0;
     bool ok = true;
-    // decode the A tile of iteration `j` (stage j % STAGES) into buffer j & 1
+    // decode k-half `half` of row r of the A tile of iteration `j` (stage j % STAGES) into buffer j & 1
     auto convert = [&](int j) -> bool {
       const int st = j % C::STAGES, cb = j & 1;
       if (!mbar_wait_warp(full_bar(st), (j / C::STAGES) & 1, abort_word, g.flag)) return false;
       if (!mbar_wait_warp(conv_free + 8 * cb, ((j >> 1) & 1) ^ 1, abort_word, g.flag)) return false;
       const uint8_t* arow = smem + st * C::STAGE + r * 128;
-      uint8_t* o0 = smem + C::ABF_OFF + cb * C::ABF + r * 128;
+      uint8_t* orow = smem + C::ABF_OFF + cb * C::ABF + half * 16384 + r * 128;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {            // 16 codes = elements 16q .. 16q+15
+      for (int qq = 0; qq < 4; ++qq) {         // 16 codes = elements 16q .. 16q+15 of the row
+        const int q = 4 * half + qq;
         const uint4 v = *reinterpret_cast<const uint4*>(arow + ((q ^ (r & 7)) << 4));
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t outw[8];
@@ -203,8 +213,7 @@ __global__ void __launch_bounds__(192, 1)
           outw[2 * k] = e4m3x2_to_f16x2(w[k] & 0xFFFF);
           outw[2 * k + 1] = e4m3x2_to_f16x2(w[k] >> 16);
         }
-        const int kk = q >> 2, c0 = 2 * (q & 3);
-        uint8_t* orow = o0 + kk * 16384;
+        const int c0 = 2 * qq;
         *reinterpret_cast<uint4*>(orow + ((c0 ^ (r & 7)) << 4)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
         *reinterpret_cast<uint4*>(orow + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(outw[4], outw[5], outw[6], outw[7]);
       }
@@ -221,20 +230,21 @@ __global__ void __launch_bounds__(192, 1)
       const int nkb = kb1 - kb0;
       first_it = it;
 #pragma unroll
-      for (int j = 0; j < BN; ++j) acc[j] = 0.f;
+      for (int j = 0; j < NCOL; ++j) acc[j] = 0.f;
       const float* sc = fa.scale + (long long)b * fa.scale_batch + (long long)mt * fa.scale_ld;
       if (nkb > 0 && !convert(first_it)) { ok = false; break; }
       for (int i = 0; i < nkb; ++i) {
         const int j = first_it + i;
         if (i + 1 < nkb && !convert(j + 1)) { ok = false; break; }
+        if (!folds) continue;
         const int pb = j & 1;
         if (!mbar_wait_warp(part_full + 8 * pb, (j >> 1) & 1, abort_word, g.flag)) { ok = false; break; }
         tc_fence_after();
         const float scl = sc[kb0 + i];
 #pragma unroll
-        for (int c = 0; c < BN / 16; ++c) {
+        for (int c = 0; c < NCOL / 16; ++c) {
           uint32_t v[16];
-          tmem_ld16(tmem + pb * BN + lane_base + 16 * c, v);
+          tmem_ld16(tmem + pb * BN + col0 + lane_base + 16 * c, v);
           tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 16; ++k) acc[16 * c + k] = fmaf(scl, __uint_as_float(v[k]), acc[16 * c + k]);
@@ -244,13 +254,14 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) break;
       it = first_it + nkb;
+      if (!folds) continue;
       const int m = mt * 128 + r;
 #pragma unroll
-      for (int c = 0; c < BN / 16; ++c) {
+      for (int c = 0; c < NCOL / 16; ++c) {
         uint32_t outv[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) outv[k] = __float_as_uint(acc[16 * c + k]);
-        gemm_store(g, m, nt * BN + 16 * c, s, b, outv);
+        gemm_store(g, m, nt * BN + col0 + 16 * c, s, b, outv);
       }
     }
   }

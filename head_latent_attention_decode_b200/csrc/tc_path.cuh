@@ -158,7 +158,7 @@ static int launch_gemm_fp8_bn(const CUtensorMap& A, const CUtensorMap& B, const 
     attr_set[dev] = true;
   }
   const int grid = fa.g.total_units < num_sms ? fa.g.total_units : num_sms;
-  launch_pdl(tc_gemm_fp8_kernel<BN>, grid, 192, C::SMEM, s, A, B, fa);
+  launch_pdl(tc_gemm_fp8_kernel<BN>, grid, 320, C::SMEM, s, A, B, fa);
   mla_count_launch(1);
   return MLA_OK;
 }
