@@ -361,7 +361,7 @@ def kernel_time(step, kernel, k, flush, stream):
     return float(np.mean(ms))
 
 
-def cpu_oracle_sample(w: wl.Workload, budget_s: float = 12.0, max_reps: int = 50) -> dict:
+def cpu_oracle_sample(w: wl.Workload, budget_s: float = 12.0, max_reps: int = 1000) -> dict:
     """The fp64 oracle, as it stands, on a bounded sample of the workload."""
     from oracle import mla_ref as ref
     from threadpoolctl import threadpool_info
