@@ -405,7 +405,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       mbar_arrive(p_full_b + 8 * sb);
       if (tr) trace[t * 16 + 5] = global_timer_ns();
     }
-    if (ok && mbar_wait_warp(o_done, (T - 1) & 1, abort_word, a.flag)) {
+    // every MMA, the last P.V included, has completed once `fin` does (waiting
+    // on o_done's parity could pass while an earlier P.V is still running)
+    if (ok && mbar_wait_warp(fin, 0, abort_word, a.flag)) {
       tc_fence_after();
       float* po = a.part_o + (unit * a.H + h) * 512 + r * 256;
       for (int c = 0; c < 16; ++c) {

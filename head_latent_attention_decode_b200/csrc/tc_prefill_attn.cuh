@@ -5,9 +5,10 @@
 //
 // One CTA per (128-query tile, head), head-major. Per 128-key tile j <= the query tile:
 //   S = Q_h . K_h^T           tcgen05, M 128 x N 128, K 192 (Q resident in smem)
-//   online softmax, one thread per query row, lazy rescale of O when the row
-//   max grows by more than 2^8; keys past the query (diagonal tile) and past
-//   the sequence are masked; P (bf16) is written into TMEM over S
+//   online softmax, one thread per query row holding its whole score row in
+//   registers, lazy rescale of O when the row max grows by more than 2^8; keys
+//   past the query (diagonal tile) and past the sequence are masked (the other
+//   tiles skip the masks); P (bf16) is written into TMEM over S
 //   O += P . V_h              tcgen05 with A = P in TMEM, M 128 x N 128, K 128,
 //                             V read MN-major from its TMA tile
 // K/V tiles stream through a 2-stage TMA ring; S runs one tile ahead of P.V.
@@ -181,16 +182,21 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait_warp(s_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sa = tmem + PA_TM_S + 128 * sb + lane_base;
-      // pass 1: row max over the valid columns
+      // the whole score row in registers (one TMEM pass)
+      uint32_t r[128];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) tmem_ld16(sa + 16 * c, r + 16 * c);
+      tmem_ld_wait();
+      // only the diagonal (or the sequence's last) tile has masked columns
+      const bool full = __all_sync(0xffffffffu, lim >= 128);
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t r[16];
-        tmem_ld16(sa + 16 * c, r);
-        tmem_ld_wait();
+        for (int j = 0; j < 128; ++j) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(r[j]));
+      } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (16 * c + j < lim) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(r[j]));
+        for (int j = 0; j < 128; ++j)
+          if (j < lim) m4[j & 3] = fmaxf(m4[j & 3], __uint_as_float(r[j]));
       }
       const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
       float alpha = 1.f;
@@ -212,20 +218,20 @@ __global__ void __launch_bounds__(192, 1)
           tmem_st16(tmem + PA_TM_O + lane_base + 16 * c, o);
         }
       }
-      // pass 2: P = 2^(s*scale - m) in bf16, written over S (chunk c of P lands on
-      // columns already consumed)
+      // P = 2^(s*scale - m) in bf16, written over S (bf16 pairs in the first 64 columns)
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t r[32], pk[16];
-        tmem_ld16(sa + 32 * c, r);
-        tmem_ld16(sa + 32 * c + 16, r + 16);
-        tmem_ld_wait();
+        uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const int col = 32 * c + j;
-          const float p0 = (col < lim) ? ex2_approx(fmaf(__uint_as_float(r[j]), a.scale_log2, nm)) : 0.f;
-          const float p1 = (col + 1 < lim) ? ex2_approx(fmaf(__uint_as_float(r[j + 1]), a.scale_log2, nm)) : 0.f;
+          float p0 = ex2_approx(fmaf(__uint_as_float(r[col]), a.scale_log2, nm));
+          float p1 = ex2_approx(fmaf(__uint_as_float(r[col + 1]), a.scale_log2, nm));
+          if (!full) {
+            p0 = col < lim ? p0 : 0.f;
+            p1 = col + 1 < lim ? p1 : 0.f;
+          }
           __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
           ps[(j >> 1) & 3] += __low2float(pb) + __high2float(pb);
           pk[j >> 1] = *reinterpret_cast<uint32_t*>(&pb);
@@ -237,7 +243,9 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(p_full_b + 8 * sb);
     }
-    if (ok && mbar_wait_warp(o_done, (T - 1) & 1, abort_word, a.flag)) {
+    // every MMA, the last P.V included, has completed once `fin` does (waiting
+    // on o_done's parity could pass while an earlier P.V is still running)
+    if (ok && mbar_wait_warp(fin, 0, abort_word, a.flag)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       bf16* o_row = a.out + (long long)qi * a.H * 128 + h * 128;
