@@ -750,7 +750,7 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
       attr[dev] = true;
     }
     mla_timer_begin("prefill_attn", s);
-    launch_pdl(tc_prefill_attn_kernel, pa.q_tiles * H, 192, PaSmem::SIZE, s, mq, mkv, mkpe, pa);
+    launch_pdl(tc_prefill_attn_kernel, pa.q_tiles * H, 320, PaSmem::SIZE, s, mq, mkv, mkpe, pa);
     mla_timer_end("prefill_attn", s);
     mla_count_launch(1);
   } else {
