@@ -111,18 +111,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full_b + 8 * i, 1);
-      mbar_init(s_free_b + 8 * i, 128);
-      mbar_init(p_full_b + 8 * i, 128);
+      mbar_init(s_free_b + 8 * i, 4);   // one arrival per softmax warp
+      mbar_init(p_full_b + 8 * i, 4);
       mbar_init(pbuf_free_b + 8 * i, 1);
       mbar_init(x_full_b + 8 * i, 1);
       mbar_init(x_free_b + 8 * i, 4);
     }
     mbar_init(o_done, 1);
     mbar_init(fin, 1);
-    mbar_init(red_b, 128);
-    mbar_init(red_b + 8, 128);
+    mbar_init(red_b, 4);
+    mbar_init(red_b + 8, 4);
     mbar_init(l_done, 4);
-    mbar_init(red2_b, 128);
+    mbar_init(red2_b, 4);
     mbar_init(fin_s, 1);
     vote[0] = -1;
     vote[1] = -1;
@@ -295,7 +295,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       for (int c = 0; c < NH / 16; ++c) tmem_ld16(tm_s + NH * sb + lane_base + 16 * c, (uint32_t*)&nxt[16 * c]);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(s_free_b + 8 * sb);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free_b + 8 * sb);
       // the peer has read what we sent for tile u - 2 out of this buffer
       if (!mbar_wait_cluster_warp(x_free_b + 8 * sb, ((u >> 1) & 1) ^ 1, abort_word, a.flag)) return false;
       if (tr0 && u < 64) trace[u * 32 + 7] = global_timer_ns();
@@ -362,7 +363,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       if (__any_sync(0xffffffffu, need) && lane == 0) vote[sb] = t;
       if (tr0 && t < 64) trace[t * 32 + 13] = global_timer_ns();
       // rendezvous of the four softmax warps on an mbarrier (a bounded wait, unlike bar.sync)
-      mbar_arrive(red_b + 8 * sb);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(red_b + 8 * sb);
       if (!mbar_wait_warp(red_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       if (tr0 && t < 64) trace[t * 32 + 3] = global_timer_ns();
       if (trace && r == 0 && lane == 0 && t < 64) trace[t * 32 + 25 + warp] = global_timer_ns();
@@ -376,7 +378,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
           const float v = warp_max_f32(valid ? cur[h] : -INFINITY);
           if (lane == 0) red[warp * NH + h] = v;
         }
-        mbar_arrive(red2_b);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(red2_b);
         if (!mbar_wait_warp(red2_b, n_slow & 1, abort_word, a.flag)) { ok = false; break; }
         ++n_slow;
 #pragma unroll
@@ -430,7 +433,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full_b + 8 * sb);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full_b + 8 * sb);
       if (tr0 && t < 64) trace[t * 32 + 4] = global_timer_ns();
       if (trace && r == 0 && lane == 0 && t < 64) trace[t * 32 + 16 + warp] = global_timer_ns();
       if (t + 1 < T && sent == t + 1) {
