@@ -248,31 +248,25 @@ class DecodeStep:
         mla.mla_decode_attn(self.layer.handle, self.q_abs, self.q_pe, self.cache, self.table,
                             self.ctx, self.max_ctx, self.out, self.ws)
 
-    # end to end through the C-ABI from pinned host buffers
+    # end to end through the C-ABI from pinned host buffers: one call copies the
+    # step's inputs in, runs RoPE tables, front-fold and attention, and copies
+    # the output back
     def e2e_setup(self):
-        pin = lambda t: t.cpu().pin_memory()
+        pin = lambda t: t.cpu().contiguous().pin_memory()
         self.h_hidden, self.h_pos, self.h_slot = pin(self.hidden), pin(self.positions), pin(self.slot)
         self.h_table, self.h_ctx = pin(self.table), pin(self.ctx)
         self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
-        self.d_bufs = [torch.empty_like(t) for t in (self.hidden, self.positions, self.slot,
-                                                     self.table, self.ctx)]
+        h = self.layer.handle
+        self.stage = torch.empty(mla.mla_decode_step_host_bytes(h, self.n, self.table.shape[1]),
+                                 dtype=torch.uint8, device="cuda")
         h2d = sum(t.numel() * t.element_size() for t in (self.h_hidden, self.h_pos, self.h_slot,
                                                          self.h_table, self.h_ctx))
         return h2d, self.h_out.numel() * self.h_out.element_size()
 
     def run_e2e(self):
-        x, p, sl, tb, cx = self.d_bufs
-        for d, h in zip(self.d_bufs, (self.h_hidden, self.h_pos, self.h_slot, self.h_table, self.h_ctx)):
-            d.copy_(h, non_blocking=True)
-        s = self.s
-        half = s.qk_rope // 2
-        cos = torch.empty((self.n, half), dtype=torch.float32, device="cuda")
-        sin = torch.empty_like(cos)
-        mla.mla_rope_cos_sin(p, s.qk_rope, s.rope_theta, cos, sin)
-        mla.mla_decode_qkv(self.layer.handle, x, cos, sin, self.cache, sl, self.q_abs, self.q_pe, self.ws)
-        mla.mla_decode_attn(self.layer.handle, self.q_abs, self.q_pe, self.cache, tb, cx,
-                            self.max_ctx, self.out, self.ws)
-        self.h_out.copy_(self.out, non_blocking=True)
+        mla.mla_decode_step_host(self.layer.handle, self.h_hidden, self.h_pos, self.h_slot, self.h_table,
+                                 self.h_ctx, self.max_ctx, self.s.rope_theta, self.cache, self.h_out,
+                                 self.stage, self.ws)
 
 
 class PrefillStep:

@@ -36,6 +36,7 @@ SYMBOLS = (
     "mla_workspace_init", "mla_read_device_flag", "mla_clear_device_flag", "mla_rope_cos_sin",
     "mla_decode_qkv", "mla_decode_attn", "mla_prefill", "mla_strerror",
     "mla_kernel_launch_count", "mla_set_kernel_timer", "mla_decode_qkv_noalloc",
+    "mla_decode_step_host_bytes", "mla_decode_step_host",
 )
 
 MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -103,6 +104,11 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_qkv_noalloc.restype = i
         L.mla_decode_qkv_noalloc.argtypes = [vp, vp, i, vp, vp, vp, i, vp, vp, vp, vp]
         L.mla_set_kernel_timer.argtypes = [ctypes.c_char_p, vp, vp]
+        L.mla_decode_step_host_bytes.restype = sz
+        L.mla_decode_step_host_bytes.argtypes = [vp, i, i]
+        L.mla_decode_step_host.restype = i
+        L.mla_decode_step_host.argtypes = [vp, vp, vp, vp, vp, i, vp, i, i, ctypes.c_double, vp, i, vp, vp, sz,
+                                           vp, sz, vp]
         _lib = L
     return _lib
 
@@ -215,6 +221,27 @@ def mla_decode_attn(handle, q_abs, q_pe, kv_cache, block_table, context_lens, ma
                                  _ptr(block_table), block_table.shape[1], _ptr(context_lens),
                                  int(max_context_len), n, _ptr(out), _ptr(head_out), _ptr(ws),
                                  _nbytes(ws), _stream(stream)), "mla_decode_attn")
+
+
+def mla_decode_step_host_bytes(handle, n: int, max_blocks_per_seq: int) -> int:
+    return int(lib().mla_decode_step_host_bytes(handle, int(n), int(max_blocks_per_seq)))
+
+
+def mla_decode_step_host(handle, hidden, positions, slot_mapping, block_table, context_lens,
+                         max_context_len, rope_theta, kv_cache, out, stage, ws, stream=None) -> None:
+    """One decode step whose inputs (hidden, positions, slot_mapping,
+    block_table, context_lens) and result (out) are host tensors, pinned for
+    asynchronous copies; kv_cache, stage and ws are device tensors. Enqueued on
+    the stream: synchronise it before reading out."""
+    for t in (hidden, positions, slot_mapping, block_table, context_lens, out):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("mla_decode_step_host: inputs and out must be contiguous host tensors")
+    n = hidden.shape[0]
+    _check(lib().mla_decode_step_host(handle, _ptr(hidden), _ptr(positions), _ptr(slot_mapping),
+                                      _ptr(block_table), block_table.shape[1], _ptr(context_lens),
+                                      int(max_context_len), n, float(rope_theta), _ptr(kv_cache),
+                                      kv_cache.shape[0], _ptr(out), _ptr(stage), _nbytes(stage), _ptr(ws),
+                                      _nbytes(ws), _stream(stream)), "mla_decode_step_host")
 
 
 def mla_prefill(handle, hidden, cos, sin, out, ws, head_out=None, kv_cache=None,

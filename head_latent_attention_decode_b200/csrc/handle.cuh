@@ -46,5 +46,22 @@ struct mla_handle {
   char* base;
   int device;
   TcState tc;
+  // mla_decode_step_host: page-locked packing buffer for the step's int32
+  // inputs, and an event marking the end of the last transfer out of it
+  void* host_pack = nullptr;
+  size_t host_pack_bytes = 0;
+  cudaEvent_t pack_done = nullptr;
+  // ... and the step captured as a CUDA graph (on the library's own stream),
+  // replayed while the call's buffers and sizes repeat
+  cudaStream_t capture_stream = nullptr;
+  cudaGraphExec_t step_exec = nullptr;
+  unsigned long long step_key[14] = {0};
+  int step_launches = 0;
+  ~mla_handle() {
+    if (pack_done) { cudaEventSynchronize(pack_done); cudaEventDestroy(pack_done); }
+    if (host_pack) cudaFreeHost(host_pack);
+    if (step_exec) cudaGraphExecDestroy(step_exec);
+    if (capture_stream) cudaStreamDestroy(capture_stream);
+  }
 };
 

@@ -233,6 +233,43 @@ int mla_decode_qkv_noalloc(mla_handle* h, const void* hidden, int n, const float
                            const float* sin, void* kv_cache, int n_blocks,
                            const int32_t* slot_mapping, void* q_abs, void* q_pe, void* stream);
 
+/* ---- one decode step from host memory ------------------------------------------ */
+
+/* Device bytes of the `stage` buffer mla_decode_step_host() needs for n tokens
+ * and block tables of max_blocks_per_seq entries: the step's inputs copied in,
+ * the cos/sin tables, q_abs, q_pe and out. 0 on invalid arguments. */
+size_t mla_decode_step_host_bytes(const mla_handle* h, int n, int max_blocks_per_seq);
+
+/* One whole decode step with its inputs and result in host memory: copies
+ * hidden, positions, slot_mapping, block_table and context_lens to the
+ * device, then runs mla_rope_cos_sin, mla_decode_qkv and mla_decode_attn (the
+ * same computation, arguments and results as those calls) and copies out back,
+ * all enqueued on `stream`. Returns once enqueued: synchronise `stream` before
+ * reading out_host. Host buffers should be page-locked (cudaHostAlloc, or
+ * torch's pin_memory) for the copies to run asynchronously; pageable memory
+ * gives the same results with blocking copies.
+ * hidden_host        host [n, D] act dtype
+ * positions_host     host [n] int32 (the position each token's RoPE uses)
+ * slot_mapping_host  host [n] int32, as in mla_decode_qkv
+ * block_table_host   host [n, max_blocks_per_seq] int32, as in mla_decode_attn
+ * context_lens_host  host [n] int32, as in mla_decode_attn
+ * rope_theta         RoPE base, as in mla_rope_cos_sin
+ * kv_cache           device, as in mla_decode_qkv (mutated in place)
+ * out_host           host [n, D] act dtype (written when the stream reaches it)
+ * stage              device buffer of mla_decode_step_host_bytes(h, n,
+ *                    max_blocks_per_seq) bytes, owned by the caller
+ * ws                 device workspace of mla_workspace_bytes(h, n, max_context_len)
+ * The four int32 arrays are packed on the host into one page-locked buffer
+ * the handle owns (allocated on the first call, regrown when a call needs
+ * more, freed by mla_destroy) and copied in one transfer; a call first waits
+ * for the previous call's transfer out of that buffer. */
+int mla_decode_step_host(mla_handle* h, const void* hidden_host, const int32_t* positions_host,
+                         const int32_t* slot_mapping_host, const int32_t* block_table_host,
+                         int max_blocks_per_seq, const int32_t* context_lens_host,
+                         int max_context_len, int n, double rope_theta, void* kv_cache,
+                         int n_blocks, void* out_host, void* stage, size_t stage_bytes, void* ws,
+                         size_t ws_bytes, void* stream);
+
 /* ---- prefill ------------------------------------------------------------------ */
 
 /* Causal prefill (context encoding) of one sequence of S tokens at positions

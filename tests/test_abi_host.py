@@ -105,6 +105,9 @@ def test_calls_reject_null_handle_and_bad_sizes(lib):
     assert lib.mla_decode_attn(None, P, P, P, 1, P, 1, P, 1, 1, P, None, P, 1 << 20, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_prefill(None, P, 1, P, P, P, None, None, 0, None, P, 1 << 20, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_workspace_bytes(None, 1, 1) == 0
+    assert lib.mla_decode_step_host_bytes(None, 1, 1) == 0
+    assert lib.mla_decode_step_host(None, P, P, P, P, 1, P, 1, 1, 10000.0, P, 1, P, P, 1 << 20, P, 1 << 20,
+                                    None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_rope_cos_sin(P, 4, 15, 10000.0, P, P, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_rope_cos_sin(P, -1, 16, 10000.0, P, P, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_rope_cos_sin(P, 4, 16, -1.0, P, P, None) == mla.MLA_ERR_INVALID_ARG
