@@ -11,7 +11,10 @@
 //   tiles skip the masks); P (bf16) is written into TMEM over S
 //   O += P . V_h              tcgen05 with A = P in TMEM, M 128 x N 128, K 128,
 //                             V read MN-major from its TMA tile
-// K/V tiles stream through a 2-stage TMA ring; S runs one tile ahead of P.V.
+// K and V tiles stream through separate 2-stage TMA rings: a K tile is released
+// as soon as its S completes, a V tile when its P.V does, so the next K tiles
+// load while the softmax runs instead of waiting for P.V. S runs one tile ahead
+// of P.V.
 // Warps 0-7 run the softmax (two threads per query row, 64 columns each, the
 // row maxima exchanged through shared memory), warp 8 issues TMA, warp 9 MMAs.
 #pragma once
@@ -30,15 +33,18 @@ struct TcPrefillAttnArgs {
 
 struct PaSmem {
   static constexpr int Q_OFF = 0;                         // 3 x [128 x 64] bf16
-  static constexpr int STAGE = 5 * 16384;                 // K: 3 x [128 x 64], V: 2 x [128 x 64]
-  static constexpr int ST_OFF = 3 * 16384;
-  static constexpr int MX_OFF = ST_OFF + 2 * STAGE;       // [2 buffers][2 halves][128] fp32 row maxima
-  static constexpr int LX_OFF = MX_OFF + 2 * 2 * 128 * 4;  // [2 halves][128] fp32 row sums
+  static constexpr int KSTAGE = 3 * 16384;                // k_nope 2 x [128 x 64], k_pe [128 x 64]
+  static constexpr int VSTAGE = 2 * 16384;                // v 2 x [128 x 64]
+  static constexpr int K_OFF = 3 * 16384;
+  static constexpr int V_OFF = K_OFF + 2 * KSTAGE;
+  static constexpr int MX_OFF = V_OFF + 2 * VSTAGE;       // [3 buffers][2 halves][128] fp32 row maxima
+  static constexpr int LX_OFF = MX_OFF + 3 * 2 * 128 * 4;  // [2 halves][128] fp32 row sums
   static constexpr int BAR_OFF = LX_OFF + 2 * 128 * 4;
   static constexpr int SIZE = 1024 + BAR_OFF + 256;
 };
-// TMEM columns: S/P buffers [0,128) [128,256), O [256,384)
-constexpr uint32_t PA_TM_S = 0, PA_TM_O = 256;
+// TMEM columns: S/P buffers [0,128) [128,256) [256,384), O [384,512)
+constexpr uint32_t PA_TM_S = 0, PA_TM_O = 384;
+constexpr int PA_SBUF = 3;   // S/P buffers: S runs up to three tiles ahead of P.V
 
 __global__ void __launch_bounds__(320, 1)
     tc_prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
@@ -48,12 +54,17 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t q_s = sbase + SM::Q_OFF, st_s = sbase + SM::ST_OFF, bar = sbase + SM::BAR_OFF;
-  const uint32_t full_b = bar, empty_b = bar + 16, s_full_b = bar + 32, p_full_b = bar + 48;
-  const uint32_t sp_empty_b = bar + 64, q_full = bar + 80, o_done = bar + 88, fin = bar + 96;
-  const uint32_t mx_b = bar + 104, lx_b = bar + 120;   // [2] half-row maxima posted; half-row sums posted
-  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 128);
-  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 132);
+  const uint32_t q_s = sbase + SM::Q_OFF, k_s = sbase + SM::K_OFF, v_s = sbase + SM::V_OFF;
+  const uint32_t bar = sbase + SM::BAR_OFF;
+  const uint32_t kfull_b = bar, kempty_b = bar + 16;                        // [2] K ring
+  const uint32_t vfull_b = bar + 32, vempty_b = bar + 48;                    // [2] V ring
+  const uint32_t s_full_b = bar + 64, p_full_b = bar + 88, sp_empty_b = bar + 112;   // [3] per S/P buffer
+  const uint32_t mx_b = bar + 136;                                           // [3] half-row maxima posted
+  // o_done[u & 1] completes with P.V(u): with S up to three tiles ahead, P.V may lag the
+  // softmax by two tiles, which one barrier's parity could not tell apart
+  const uint32_t q_full = bar + 160, o_done = bar + 168, fin = bar + 184, lx_b = bar + 192;
+  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 224);
+  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 228);
 
   // head-major order so that the CTAs in flight share one or two heads' K/V in
   // L2; within a head the heaviest query tiles (causal work grows with the
@@ -65,8 +76,12 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(full_b + 8 * i, 1);
-      mbar_init(empty_b + 8 * i, 1);
+      mbar_init(kfull_b + 8 * i, 1);
+      mbar_init(kempty_b + 8 * i, 1);
+      mbar_init(vfull_b + 8 * i, 1);
+      mbar_init(vempty_b + 8 * i, 1);
+    }
+    for (int i = 0; i < PA_SBUF; ++i) {
       mbar_init(s_full_b + 8 * i, 1);
       mbar_init(p_full_b + 8 * i, 8);   // one arrival per softmax warp
       mbar_init(mx_b + 8 * i, 8);
@@ -74,6 +89,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(q_full, 1);
     mbar_init(o_done, 1);
+    mbar_init(o_done + 8, 1);
     mbar_init(fin, 1);
     mbar_init(lx_b, 8);
     *abort_word = 0;
@@ -92,25 +108,54 @@ __global__ void __launch_bounds__(320, 1)
       prefetch_tmap(&tm_kv);
       mbar_arrive_expect_tx(q_full, 3 * 16384);
       for (int j = 0; j < 3; ++j) tma_load_3d(q_s + j * 16384, &tm_q, q_full, h * 192 + 64 * j, qt * 128, 0);
-      int t = 0;
-      for (; t < T; ++t) {
-        const int st = t & 1;
-        if (!mbar_wait(empty_b + 8 * st, ((t >> 1) & 1) ^ 1, abort_word, a.flag)) break;
-        const uint32_t dst = st_s + st * SM::STAGE;
-        mbar_arrive_expect_tx(full_b + 8 * st, 5 * 16384);
-        tma_load_3d(dst, &tm_kv, full_b + 8 * st, h * 256, t * 128, 0);               // k_nope 0..63
-        tma_load_3d(dst + 16384, &tm_kv, full_b + 8 * st, h * 256 + 64, t * 128, 0);  // k_nope 64..127
-        tma_load_3d(dst + 2 * 16384, &tm_kpe, full_b + 8 * st, 0, t * 128, 0);        // k_pe
-        tma_load_3d(dst + 3 * 16384, &tm_kv, full_b + 8 * st, h * 256 + 128, t * 128, 0);  // v 0..63
-        tma_load_3d(dst + 4 * 16384, &tm_kv, full_b + 8 * st, h * 256 + 192, t * 128, 0);  // v 64..127
+      // K(t) needs S(t-2) done, V(t) needs P.V(t-2) done: issue each as soon as its slot frees
+      int kt = 0, vt = 0;
+      bool ok = true;
+      uint64_t t_last = global_timer_ns();
+      while (ok && (kt < T || vt < T)) {
+        bool did = false;
+        if (kt < T && mbar_test(kempty_b + 8 * (kt & 1), ((kt >> 1) & 1) ^ 1)) {
+          const uint32_t kb = kfull_b + 8 * (kt & 1), dst = k_s + (kt & 1) * SM::KSTAGE;
+          mbar_arrive_expect_tx(kb, 3 * 16384);
+          tma_load_3d(dst, &tm_kv, kb, h * 256, kt * 128, 0);               // k_nope 0..63
+          tma_load_3d(dst + 16384, &tm_kv, kb, h * 256 + 64, kt * 128, 0);  // k_nope 64..127
+          tma_load_3d(dst + 2 * 16384, &tm_kpe, kb, 0, kt * 128, 0);        // k_pe
+          ++kt;
+          did = true;
+        }
+        if (vt < kt && mbar_test(vempty_b + 8 * (vt & 1), ((vt >> 1) & 1) ^ 1)) {
+          const uint32_t vb = vfull_b + 8 * (vt & 1), dst = v_s + (vt & 1) * SM::VSTAGE;
+          mbar_arrive_expect_tx(vb, 2 * 16384);
+          tma_load_3d(dst, &tm_kv, vb, h * 256 + 128, vt * 128, 0);           // v 0..63
+          tma_load_3d(dst + 16384, &tm_kv, vb, h * 256 + 192, vt * 128, 0);   // v 64..127
+          ++vt;
+          did = true;
+        }
+        if (did) {
+          t_last = global_timer_ns();
+        } else if (*abort_word) {
+          ok = false;
+        } else if (global_timer_ns() - t_last > WAIT_LIMIT_NS) {
+          *abort_word = 1;
+          set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT);
+          ok = false;
+        } else {
+          __nanosleep(32);
+        }
       }
+      // drain the loads still in flight
       {
         const uint64_t t0 = global_timer_ns();
         while (!mbar_try_wait(q_full, 0)) if (global_timer_ns() - t0 > WAIT_LIMIT_NS) break;
       }
-      for (int u = (t > 2 ? t - 2 : 0); u < t; ++u) {
+      for (int u = (kt > 2 ? kt - 2 : 0); u < kt; ++u) {
         const uint64_t t1 = global_timer_ns();
-        while (!mbar_try_wait(full_b + 8 * (u & 1), (u >> 1) & 1))
+        while (!mbar_try_wait(kfull_b + 8 * (u & 1), (u >> 1) & 1))
+          if (global_timer_ns() - t1 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
+      }
+      for (int u = (vt > 2 ? vt - 2 : 0); u < vt; ++u) {
+        const uint64_t t1 = global_timer_ns();
+        while (!mbar_try_wait(vfull_b + 8 * (u & 1), (u >> 1) & 1))
           if (global_timer_ns() - t1 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
       }
     }
@@ -121,52 +166,67 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t idesc_o = idesc_bf16(128, 128, 1);
       bool ok = mbar_wait(q_full, 0, abort_word, a.flag);
       // descriptors built once; buffers and k-steps add their byte offset >> 4
-      const uint64_t d_q = sdesc_sw128(q_s), d_k = sdesc_sw128(st_s);
-      const uint64_t d_v = sdesc_sw128_mn(st_s + 3 * 16384, 16384);
+      const uint64_t d_q = sdesc_sw128(q_s), d_k = sdesc_sw128(k_s);
+      const uint64_t d_v = sdesc_sw128_mn(v_s, 16384);
       int next_s = 0, next_o = 0;
-      uint64_t t_last = global_timer_ns();
+      uint32_t idle = 0;
+      uint64_t t_idle = 0;
       while (ok && next_o < T) {
         bool did = false;
-        if (next_s < T && next_s < next_o + 2) {
-          const int t = next_s, st = t & 1;
-          if (mbar_test(full_b + 8 * st, (t >> 1) & 1) && mbar_test(sp_empty_b + 8 * st, ((t >> 1) & 1) ^ 1)) {
+        // P.V first: the S buffer it frees is what lets S run ahead
+        if (next_o < next_s) {
+          const int u = next_o, sb = u % PA_SBUF, vs = u & 1;
+          if (mbar_test(p_full_b + 8 * sb, (u / PA_SBUF) & 1) && mbar_test(vfull_b + 8 * vs, (u >> 1) & 1)) {
             tc_fence_after();
-            const uint64_t dk = d_k + (uint64_t)(st * (SM::STAGE / 16));
-#pragma unroll
-            for (int j = 0; j < 3; ++j)
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16(tmem + PA_TM_S + 128 * st, d_q + (j * 16384 + 32 * k) / 16, dk + (j * 16384 + 32 * k) / 16,
-                         idesc_s, (j > 0 || k > 0) ? 1u : 0u);
-            mma_commit(s_full_b + 8 * st);
-            ++next_s;
-            did = true;
-          }
-        }
-        if (!did && next_o < next_s) {
-          const int u = next_o, st = u & 1;
-          if (mbar_test(p_full_b + 8 * st, (u >> 1) & 1)) {
-            tc_fence_after();
-            const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
+            const uint64_t dv = d_v + (uint64_t)(vs * (SM::VSTAGE / 16));
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              mma_bf16_ts(tmem + PA_TM_O, tmem + PA_TM_S + 128 * st + 8 * k, dv + 2048 * k / 16, idesc_o,
+              mma_bf16_ts(tmem + PA_TM_O, tmem + PA_TM_S + 128 * sb + 8 * k, dv + 2048 * k / 16, idesc_o,
                           (u > 0 || k > 0) ? 1u : 0u);
-            mma_commit(o_done);
-            mma_commit(sp_empty_b + 8 * st);
-            mma_commit(empty_b + 8 * st);
+            mma_commit(o_done + 8 * (u & 1));
+            mma_commit(sp_empty_b + 8 * sb);
+            mma_commit(vempty_b + 8 * vs);
             ++next_o;
             did = true;
           }
         }
+        if (!did && next_s < T && next_s < next_o + PA_SBUF) {
+          const int t = next_s, sb = t % PA_SBUF, ks = t & 1;
+          if (mbar_test(kfull_b + 8 * ks, (t >> 1) & 1) &&
+              mbar_test(sp_empty_b + 8 * sb, ((t / PA_SBUF) & 1) ^ 1)) {
+            tc_fence_after();
+            const uint64_t dk = d_k + (uint64_t)(ks * (SM::KSTAGE / 16));
+#pragma unroll
+            for (int j = 0; j < 3; ++j)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_bf16(tmem + PA_TM_S + 128 * sb, d_q + (j * 16384 + 32 * k) / 16, dk + (j * 16384 + 32 * k) / 16,
+                         idesc_s, (j > 0 || k > 0) ? 1u : 0u);
+            mma_commit(s_full_b + 8 * sb);
+            mma_commit(kempty_b + 8 * ks);
+            ++next_s;
+            did = true;
+          }
+        }
+        // the clock is read only while idle: first idle pass, then every 64th; an
+        // idle pass backs off so that the polling does not take issue slots from
+        // the softmax warps sharing this scheduler
         if (did) {
-          t_last = global_timer_ns();
+          idle = 0;
         } else if (*abort_word) {
           ok = false;
-        } else if (global_timer_ns() - t_last > WAIT_LIMIT_NS) {
-          *abort_word = 1;
-          set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT);
-          ok = false;
+        } else {
+          if ((++idle & 63) == 1) {
+            const uint64_t now = global_timer_ns();
+            if (idle == 1) {
+              t_idle = now;
+            } else if (now - t_idle > WAIT_LIMIT_NS) {
+              *abort_word = 1;
+              set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT);
+              ok = false;
+            }
+          }
+          __nanosleep(32);
         }
       }
       mma_commit(fin);
@@ -179,16 +239,16 @@ __global__ void __launch_bounds__(320, 1)
     const int row = threadIdx.x & 127, half = threadIdx.x >> 7;
     const int qi = qt * 128 + row;                // this thread's query position
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    float* mx = (float*)(smem + SM::MX_OFF);      // [sb][half][row]
+    float* mx = (float*)(smem + SM::MX_OFF);      // [sb][half][row], sb = S/P buffer
     float* lx = (float*)(smem + SM::LX_OFF);      // [half][row]
     float m_ref = -INFINITY, l = 0.f;             // the same reference in both threads of a row
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
-      const int sb = t & 1;
+      const int sb = t % PA_SBUF, ph = (t / PA_SBUF) & 1;
       // keys k0 .. k0+127; key k valid iff k <= qi and k < S
       const int k0 = t * 128;
       const int lim = min(qi, a.S - 1) - k0 + 1 - 64 * half;   // valid columns of this half: [0, lim)
-      if (!mbar_wait_warp(s_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (!mbar_wait_warp(s_full_b + 8 * sb, ph, abort_word, a.flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sa = tmem + PA_TM_S + 128 * sb + lane_base;
       // this half of the score row in registers
@@ -211,7 +271,7 @@ __global__ void __launch_bounds__(320, 1)
       mx[(sb * 2 + half) * 128 + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       __syncwarp();
       if (lane == 0) mbar_arrive(mx_b + 8 * sb);
-      if (!mbar_wait_warp(mx_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (!mbar_wait_warp(mx_b + 8 * sb, ph, abort_word, a.flag)) { ok = false; break; }
       const float mt = fmaxf(mx[(sb * 2) * 128 + row], mx[(sb * 2 + 1) * 128 + row]) * a.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -221,7 +281,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
       if (__any_sync(0xffffffffu, rescale) && t >= 1) {
-        if (!mbar_wait_warp(o_done, (t - 1) & 1, abort_word, a.flag)) { ok = false; break; }
+        if (!mbar_wait_warp(o_done + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
         tc_fence_after();
         for (int c = 0; c < 4; ++c) {   // this half's 64 columns of O
           uint32_t o[16];
