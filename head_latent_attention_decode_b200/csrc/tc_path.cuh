@@ -496,7 +496,6 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
                                 char* ws, size_t tc_off, cudaStream_t s) {
   const mla_config& c = h->cfg;
   const WeightLayout& L = h->L;
-  const TcState& T = h->tc;
   const TcDecodeWs W = tc_decode_ws(h, n);
   char* tw = ws + tc_off;
   int* flag = (int*)ws;
@@ -658,7 +657,6 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
                                  int max_ctx, int n, void* out, void* head, char* ws, size_t tc_off,
                                  cudaStream_t s, float* part_o, float* part_ml, int splits, bf16* o_lat) {
   const mla_config& c = h->cfg;
-  const TcState& T = h->tc;
   const TcDecodeWs W = tc_decode_ws(h, n);
   char* tw = ws + tc_off;
   int* flag = (int*)ws;
