@@ -64,6 +64,14 @@ def test_v2lite_bf16_prefill_small():
     run_prefill(V2LITE_PREFILL, S=200)
 
 
+@pytest.mark.parametrize("S", [1, 128, 129, 256])
+def test_v2lite_bf16_prefill_tile_edges(S):
+    """The tensor-core attention's degenerate sizes: one token (a single
+    diagonal tile with one key), exactly one query tile, one row into a second
+    tile, and an exact multiple of the tile."""
+    run_prefill(V2LITE_PREFILL, S=S, with_cache=True)
+
+
 def test_v3_bf16_prefill_small():
     run_prefill(wl.WORKLOADS["v3_prefill_bf16"], S=300, with_cache=True)
 
