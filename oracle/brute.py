@@ -28,11 +28,12 @@ def _rms(v, g, eps):
     return [v[i] * r * g[i] for i in range(len(v))]
 
 
-def _rope(v, pos, theta):
+def _rope(v, pos, theta, inv_freq=None):
     d = len(v)
     out = list(v)
     for i in range(d // 2):
-        phi = pos * theta ** (-2.0 * i / d)
+        f = theta ** (-2.0 * i / d) if inv_freq is None else float(inv_freq[i])
+        phi = pos * f
         a, b = v[2 * i], v[2 * i + 1]
         out[2 * i] = a * math.cos(phi) - b * math.sin(phi)
         out[2 * i + 1] = a * math.sin(phi) + b * math.cos(phi)
@@ -40,9 +41,12 @@ def _rope(v, pos, theta):
 
 
 def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens,
-                slot_mapping, layout=0):
+                slot_mapping, layout=0, input_norm_w=None, inv_freq=None):
     """One whole decode step, loops only.
 
+    input_norm_w: optional input RMSNorm gamma [hidden] applied to each token
+    first (eps = norm_eps); inv_freq: optional RoPE frequency table [d_r/2]
+    replacing theta^(-2i/d_r).
     cache_rows: list of flat cache rows (lists of R floats), mutated copy returned.
     Returns (out [n][hidden], head_out [n][H][d_v], q_abs [n][H][r_kv],
     q_pe [n][H][d_r], new cache_rows).
@@ -54,6 +58,8 @@ def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens
     q_abs_all, q_pe_all = [], []
     for t, x in enumerate(hidden):
         x = [float(v) for v in x]
+        if input_norm_w is not None:
+            x = _rms(x, [float(g) for g in input_norm_w], cfg.norm_eps)
         pos = int(positions[t])
         if cfg.q_lora_rank:
             ql = _rms(_vecmat(x, _mat(W["wq_a"])), [float(g) for g in W["q_norm_w"]], cfg.norm_eps)
@@ -62,11 +68,11 @@ def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens
             q = _vecmat(x, _mat(W["wq_b"]))
         kv = _vecmat(x, _mat(W["wkv_a"]))
         c = _rms(kv[:rkv], [float(g) for g in W["kv_norm_w"]], cfg.norm_eps)
-        kpe = _rope(kv[rkv:], pos, cfg.rope_theta)
+        kpe = _rope(kv[rkv:], pos, cfg.rope_theta, inv_freq)
         q_abs_t, q_pe_t = [], []
         for h in range(H):
             qh = q[h * (dn + dr):(h + 1) * (dn + dr)]
-            qn, qp = qh[:dn], _rope(qh[dn:], pos, cfg.rope_theta)
+            qn, qp = qh[:dn], _rope(qh[dn:], pos, cfg.rope_theta, inv_freq)
             # absorption through the nope columns of head h of wkv_b
             qa = [sum(qn[p] * wkv_b[cc][h * (dn + dv) + p] for p in range(dn)) for cc in range(rkv)]
             q_abs_t.append(qa)

@@ -50,13 +50,17 @@ def rope_inv_freq(rope_dim, theta):
     return theta ** (-2.0 * i / rope_dim)
 
 
-def rope_cos_sin(positions, rope_dim, theta):
+def rope_cos_sin(positions, rope_dim, theta, inv_freq=None):
     """Half-width tables [n, d_r/2] of cos/sin(pos * inv_freq_i).
 
     Half width as "MLA Decode QKV Kernel API Reference", Parameters (cos, sin:
-    [n_tokens, qk_rope_dim // 2]).
+    [n_tokens, qk_rope_dim // 2]). inv_freq, when given, is a precomputed
+    [d_r/2] table used as is ("Struct MlaWeights", field yarn_inv_freq: a
+    precomputed YaRN inv_freq table [rotary_dim/2]; NULL selects the standard
+    theta computation), and theta is then unused.
     """
-    phi = np.asarray(positions, np.float64)[:, None] * rope_inv_freq(rope_dim, theta)[None, :]
+    f = rope_inv_freq(rope_dim, theta) if inv_freq is None else np.asarray(inv_freq, np.float64)
+    phi = np.asarray(positions, np.float64)[:, None] * f[None, :]
     return np.cos(phi), np.sin(phi)
 
 
@@ -264,13 +268,27 @@ def absorb(q_nope, w_uk):
     return np.einsum("thp,hpc->thc", q_nope, w_uk)
 
 
-def decode_qkv(cfg, W, hidden, cos, sin, kv_cache, slot_mapping, row_layout=LATENT_FIRST):
+def input_norm(cfg, hidden, input_norm_w):
+    """The layer's input RMSNorm, rms_norm(x, input_norm_w) with eps = norm_eps.
+
+    "MLA Decode QKV Kernel API Reference", Parameters (input_norm_w: [1,
+    hidden] fp32, optional; when given, the layer's input RMSNorm is folded into
+    the hidden load). The page names no separate epsilon, so the reading is the
+    kernel's norm_eps.
+    """
+    return rms_norm(hidden, input_norm_w, cfg.norm_eps)
+
+
+def decode_qkv(cfg, W, hidden, cos, sin, kv_cache, slot_mapping, row_layout=LATENT_FIRST, input_norm_w=None):
     """The decode front-fold: (q_abs [n,H,r_kv], q_pe [n,H,d_r], new kv_cache).
 
     "MLA Decode QKV Kernel API Reference", mla_decode_qkv: query and KV
     projections, both RMSNorms, interleaved RoPE, absorption of the query into
     the latent space, and the scatter of this step's row into the paged cache.
+    With input_norm_w the hidden states are first RMS-normalised (input_norm).
     """
+    if input_norm_w is not None:
+        hidden = input_norm(cfg, hidden, input_norm_w)
     q_nope, q_pe = decode_q(cfg, W, hidden, cos, sin)
     c, k_pe = kv_projection(cfg, W, hidden, cos, sin)
     w_uk, _ = split_wkv_b(W["wkv_b"], cfg.n_heads, cfg.qk_nope, cfg.v_dim)

@@ -56,6 +56,62 @@ def test_decode_matches_brute_force(shape, layout):
     np.testing.assert_allclose(out, np.array(b_out), rtol=0, atol=1e-12)
 
 
+def _yarn_like_inv_freq(rope_dim, theta=10000.0, factor=8.0):
+    """A frequency table of the YaRN kind for the pins: the low frequencies
+    divided by `factor`, the high ones kept, a linear ramp in between (any
+    positive table serves; only its use as given is pinned)."""
+    i = np.arange(rope_dim // 2, dtype=np.float64)
+    base = theta ** (-2.0 * i / rope_dim)
+    ramp = np.clip((i - 0.25 * len(i)) / max(0.5 * len(i), 1.0), 0.0, 1.0)
+    return base * (1.0 - ramp) + base / factor * ramp
+
+
+@pytest.mark.parametrize("shape", [SMALL, SMALL_NOQ])
+def test_decode_with_input_norm_and_inv_freq_matches_brute_force(shape):
+    """The optional input RMSNorm ("MLA Decode QKV Kernel API Reference",
+    input_norm_w) and a precomputed RoPE frequency table ("Struct MlaWeights",
+    yarn_inv_freq) against the literal loops."""
+    W, inp, _, _ = _decode_case(shape, 11)
+    rng = np.random.default_rng(11)
+    g_in = 1.0 + rng.uniform(-0.3, 0.3, shape.hidden)
+    f = _yarn_like_inv_freq(shape.qk_rope)
+    cos, sin = ref.rope_cos_sin(inp.positions, shape.qk_rope, shape.rope_theta, inv_freq=f)
+    q_abs, q_pe, cache = ref.decode_qkv(shape, W, inp.hidden, cos, sin, inp.cache, inp.slot_mapping,
+                                        input_norm_w=g_in)
+    out, head_out = ref.decode_attn(shape, W, q_abs, q_pe, cache, inp.block_table, inp.context_lens)
+    b_out, b_head, b_qabs, b_qpe, b_rows = brute.decode_step(
+        shape, W, inp.hidden, inp.positions, inp.cache.reshape(-1, shape.kv_row_dim).tolist(),
+        inp.block_table.tolist(), inp.context_lens, inp.slot_mapping, input_norm_w=g_in, inv_freq=f)
+    np.testing.assert_allclose(q_abs, np.array(b_qabs), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(q_pe, np.array(b_qpe), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(cache.reshape(-1, shape.kv_row_dim), np.array(b_rows), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out, np.array(b_out), rtol=0, atol=1e-12)
+
+
+def test_input_norm_removes_the_input_scale():
+    """RMSNorm makes the front-fold blind to a positive scale of x (up to eps):
+    scaling the hidden states by 3.7 changes nothing, whereas without the
+    norm the unnormed k_pe scales with x."""
+    W, inp, cos, sin = _decode_case(SMALL, 12)
+    g_in = 1.0 + np.random.default_rng(12).uniform(-0.3, 0.3, SMALL.hidden)
+    a = ref.decode_qkv(SMALL, W, inp.hidden, cos, sin, inp.cache, inp.slot_mapping, input_norm_w=g_in)
+    b = ref.decode_qkv(SMALL, W, 3.7 * inp.hidden, cos, sin, inp.cache, inp.slot_mapping, input_norm_w=g_in)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, rtol=1e-6, atol=1e-9)
+    c = ref.decode_qkv(SMALL, W, 3.7 * inp.hidden, cos, sin, inp.cache, inp.slot_mapping)
+    d = ref.decode_qkv(SMALL, W, inp.hidden, cos, sin, inp.cache, inp.slot_mapping)
+    assert np.max(np.abs(c[2] - d[2])) > 1e-3
+
+
+def test_inv_freq_table_of_plain_theta_reproduces_theta():
+    pos = np.array([0, 1, 7, 4095])
+    c0, s0 = ref.rope_cos_sin(pos, 64, 10000.0)
+    i = np.arange(32)
+    c1, s1 = ref.rope_cos_sin(pos, 64, 1.0, inv_freq=10000.0 ** (-i / 32.0))
+    np.testing.assert_allclose(c0, c1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s0, s1, rtol=0, atol=1e-12)
+
+
 @pytest.mark.parametrize("shape", [SMALL, SMALL_NOQ])
 def test_prefill_matches_brute_force(shape):
     W = _weights(shape, 3)
@@ -428,6 +484,23 @@ def test_planted_wkv_b_grouping_is_caught(monkeypatch):
         return k, v
     monkeypatch.setattr(ref, "split_wkv_b", grouped_wrong)
     assert _brute_decode_mismatch(SMALL) > 1e-6
+
+
+def test_planted_input_norm_without_gamma_is_caught(monkeypatch):
+    W, inp, cos, sin = _decode_case(SMALL, 13)
+    g_in = 1.0 + np.random.default_rng(13).uniform(-0.3, 0.3, SMALL.hidden)
+    flat = inp.cache.reshape(-1, SMALL.kv_row_dim).tolist()
+
+    def mismatch():
+        _, q_pe, cache = ref.decode_qkv(SMALL, W, inp.hidden, cos, sin, inp.cache, inp.slot_mapping,
+                                        input_norm_w=g_in)
+        b = brute.decode_step(SMALL, W, inp.hidden, inp.positions, flat, inp.block_table.tolist(),
+                              inp.context_lens, inp.slot_mapping, input_norm_w=g_in)
+        return max(np.max(np.abs(q_pe - np.array(b[3]))),
+                   np.max(np.abs(cache.reshape(-1, SMALL.kv_row_dim) - np.array(b[4]))))
+    assert mismatch() < 1e-12
+    monkeypatch.setattr(ref, "input_norm", lambda cfg, x, g: ref.rms_norm(x, np.ones_like(g), cfg.norm_eps))
+    assert mismatch() > 1e-6
 
 
 def test_planted_normed_k_pe_is_caught(monkeypatch):
