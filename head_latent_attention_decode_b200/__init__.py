@@ -36,7 +36,7 @@ SYMBOLS = (
     "mla_workspace_init", "mla_read_device_flag", "mla_clear_device_flag", "mla_rope_cos_sin",
     "mla_decode_qkv", "mla_decode_attn", "mla_prefill", "mla_strerror",
     "mla_kernel_launch_count", "mla_set_kernel_timer", "mla_decode_qkv_noalloc",
-    "mla_decode_step_host_bytes", "mla_decode_step_host",
+    "mla_decode_step_host_bytes", "mla_decode_step_host", "mla_rope_cos_sin_inv_freq",
 )
 
 MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -104,6 +104,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_qkv_noalloc.restype = i
         L.mla_decode_qkv_noalloc.argtypes = [vp, vp, i, vp, vp, vp, i, vp, vp, vp, vp]
         L.mla_set_kernel_timer.argtypes = [ctypes.c_char_p, vp, vp]
+        L.mla_rope_cos_sin_inv_freq.restype = i
+        L.mla_rope_cos_sin_inv_freq.argtypes = [vp, i, i, vp, vp, vp, vp]
         L.mla_decode_step_host_bytes.restype = sz
         L.mla_decode_step_host_bytes.argtypes = [vp, i, i]
         L.mla_decode_step_host.restype = i
@@ -193,6 +195,13 @@ def mla_rope_cos_sin(positions: torch.Tensor, qk_rope: int, theta: float, cos: t
                      sin: torch.Tensor, stream=None) -> None:
     _check(lib().mla_rope_cos_sin(_ptr(positions), positions.numel(), qk_rope, float(theta),
                                   _ptr(cos), _ptr(sin), _stream(stream)), "mla_rope_cos_sin")
+
+
+def mla_rope_cos_sin_inv_freq(positions: torch.Tensor, qk_rope: int, inv_freq: torch.Tensor, cos: torch.Tensor,
+                              sin: torch.Tensor, stream=None) -> None:
+    """RoPE tables from a precomputed frequency table (e.g. YaRN's) [qk_rope/2] fp32."""
+    _check(lib().mla_rope_cos_sin_inv_freq(_ptr(positions), positions.numel(), qk_rope, _ptr(inv_freq),
+                                           _ptr(cos), _ptr(sin), _stream(stream)), "mla_rope_cos_sin_inv_freq")
 
 
 def mla_decode_qkv(handle, hidden, cos, sin, kv_cache, slot_mapping, q_abs, q_pe, ws,

@@ -106,7 +106,7 @@ static WeightLayout make_layout(const mla_config* c) {
 // [0, 256): device flag (int32 at 0) and counters. Then decode and prefill
 // scratch share one region (calls on one workspace are stream-ordered).
 struct WsLayout {
-  size_t Y1, qn, Q, part_o, part_ml, o_lat, head;             // decode
+  size_t Y1, qn, Q, part_o, part_ml, o_lat, head, xn;         // decode
   size_t pY1, pqn, pQ, pcn, pkpe, pKV, phead;                  // prefill
   size_t tc;                                                   // tensor-core path scratch
   size_t total;
@@ -134,6 +134,7 @@ static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
   W.part_ml = put((size_t)n * W.splits * H * 2 * 4);
   W.o_lat = put((size_t)n * H * rkv * a);
   W.head = put((size_t)n * H * dv * a);
+  W.xn = put((size_t)n * c->hidden * a);
   W.tc = put(tc_decode_ws_bytes(h, n, max_ctx));
   const size_t dec_end = off;
   off = 256;
@@ -352,11 +353,22 @@ int mla_rope_cos_sin(const int32_t* positions, int n, int qk_rope, double theta,
   return cuda_status();
 }
 
+int mla_rope_cos_sin_inv_freq(const int32_t* positions, int n, int qk_rope, const float* inv_freq,
+                              float* cos_out, float* sin_out, void* stream) {
+  if (n < 0 || qk_rope <= 0 || qk_rope % 2) return MLA_ERR_INVALID_ARG;
+  if (n == 0) return MLA_OK;
+  if (!positions || !inv_freq || !cos_out || !sin_out) return MLA_ERR_INVALID_ARG;
+  const long long total = (long long)n * (qk_rope / 2);
+  const int blocks = (int)(cdiv(total, 256) > 4096 ? 4096 : cdiv(total, 256));
+  rope_table_freq_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(positions, n, qk_rope, inv_freq, cos_out, sin_out);
+  count_launch();
+  return cuda_status();
+}
+
 int mla_decode_qkv(mla_handle* h, const void* hidden, int n, const float* cos, const float* sin,
                    void* kv_cache, int n_blocks, const int32_t* slot_mapping, void* q_abs, void* q_pe,
                    const float* input_norm_w, void* ws, size_t ws_bytes, void* stream) {
   if (!h || n < 0 || n_blocks < 0) return MLA_ERR_INVALID_ARG;
-  if (input_norm_w) return MLA_ERR_UNSUPPORTED;
   if (n == 0) return MLA_OK;
   if (!hidden || !cos || !sin || !kv_cache || !slot_mapping || !q_abs || !q_pe || !ws)
     return MLA_ERR_INVALID_ARG;
@@ -370,6 +382,14 @@ int mla_decode_qkv(mla_handle* h, const void* hidden, int n, const float* cos, c
   const int H = c->n_heads, dn = c->qk_nope, dr = c->qk_rope, rkv = c->kv_lora_rank, D = c->hidden;
   const int rq = c->q_lora_rank;
   const int ta = acode(h), tw = wcode(h);
+  if (input_norm_w) {
+    // 0. the layer's input RMSNorm into the workspace; the path reads that instead
+    void* xn = wsb + W.xn;
+    if (ta == 0) input_rmsnorm_kernel<float><<<n, 256, 0, s>>>((const float*)hidden, input_norm_w, D, c->norm_eps, (float*)xn);
+    else input_rmsnorm_kernel<bf16><<<n, 256, 0, s>>>((const bf16*)hidden, input_norm_w, D, c->norm_eps, (bf16*)xn);
+    count_launch();
+    hidden = xn;
+  }
   if (tc_decode_qkv_supported(h, n)) {
     const int r = tc_decode_qkv(h, hidden, n, cos, sin, kv_cache, n_blocks, slot_mapping, q_abs, q_pe,
                                 wsb, W.tc, s);

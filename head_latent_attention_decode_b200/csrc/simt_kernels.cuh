@@ -482,4 +482,38 @@ __global__ void rope_table_kernel(const int* pos, int n, int d_r, double theta, 
   }
 }
 
+// RoPE tables from a given frequency table: angle = pos * inv_freq[i], the
+// product and the cosine / sine in fp64, rounded once to fp32 ("Struct
+// MlaWeights", yarn_inv_freq: a precomputed [rotary_dim/2] table).
+__global__ void rope_table_freq_kernel(const int* pos, int n, int d_r, const float* inv_freq, float* cs, float* sn) {
+  const int half = d_r / 2;
+  const long long total = (long long)n * half;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(idx / half), i = (int)(idx % half);
+    const double phi = (double)pos[t] * (double)inv_freq[i];
+    double sv, cv;
+    sincos(phi, &sv, &cv);
+    cs[idx] = (float)cv;
+    sn[idx] = (float)sv;
+  }
+}
+
+// The layer's input RMSNorm, one CTA per token: xn = x * rsqrt(mean(x^2) + eps)
+// * gamma in the activation dtype ("MLA Decode QKV Kernel API Reference",
+// input_norm_w: the input RMSNorm folded into the hidden load).
+template <typename T>
+__global__ void __launch_bounds__(256) input_rmsnorm_kernel(const T* x, const float* gamma, int D, float eps, T* xn) {
+  __shared__ float red[32];
+  const T* xr = x + (long long)blockIdx.x * D;
+  T* yr = xn + (long long)blockIdx.x * D;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    const float v = to_f32(xr[i]);
+    ss += v * v;
+  }
+  const float r = rsqrtf(block_sum(ss, red) / (float)D + eps);
+  for (int i = threadIdx.x; i < D; i += blockDim.x) yr[i] = from_f32<T>(to_f32(xr[i]) * r * gamma[i]);
+}
+
 }  // namespace mla

@@ -9,7 +9,7 @@ import numpy as np
 import torch
 
 from . import (MLA_ROW_LATENT_FIRST, make_config, mla_decode_attn, mla_decode_qkv, mla_destroy,
-               mla_init_weights, mla_prefill, mla_rope_cos_sin, mla_weights_bytes,
+               mla_init_weights, mla_prefill, mla_rope_cos_sin, mla_rope_cos_sin_inv_freq, mla_weights_bytes,
                mla_workspace_bytes, mla_workspace_init)
 
 ACT_TORCH = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -64,15 +64,20 @@ class MlaLayer:
             mla_workspace_init(self.ws)
         return self.ws
 
-    def rope(self, positions: torch.Tensor):
+    def rope(self, positions: torch.Tensor, inv_freq: torch.Tensor | None = None):
+        """cos/sin [n, qk_rope/2] fp32 of the positions; inv_freq (device fp32
+        [qk_rope/2], e.g. a YaRN table) replaces theta^(-2i/qk_rope)."""
         n = positions.numel()
         half = self.shape.qk_rope // 2
         cos = torch.empty((n, half), dtype=torch.float32, device=self.device)
         sin = torch.empty((n, half), dtype=torch.float32, device=self.device)
-        mla_rope_cos_sin(positions, self.shape.qk_rope, self.shape.rope_theta, cos, sin)
+        if inv_freq is None:
+            mla_rope_cos_sin(positions, self.shape.qk_rope, self.shape.rope_theta, cos, sin)
+        else:
+            mla_rope_cos_sin_inv_freq(positions, self.shape.qk_rope, inv_freq, cos, sin)
         return cos, sin
 
-    def decode_qkv(self, hidden, cos, sin, kv_cache, slot_mapping, q_abs=None, q_pe=None):
+    def decode_qkv(self, hidden, cos, sin, kv_cache, slot_mapping, q_abs=None, q_pe=None, input_norm_w=None):
         s = self.shape
         n = hidden.shape[0]
         if q_abs is None:
@@ -81,7 +86,8 @@ class MlaLayer:
             q_pe = torch.empty((n, s.n_heads, s.qk_rope), dtype=self.act, device=self.device)
         ws = self.ws if self.ws is not None and self.ws.numel() >= mla_workspace_bytes(
             self.handle, max(n, 1), 1) else self.workspace(n, 1)
-        mla_decode_qkv(self.handle, hidden, cos, sin, kv_cache, slot_mapping, q_abs, q_pe, ws)
+        mla_decode_qkv(self.handle, hidden, cos, sin, kv_cache, slot_mapping, q_abs, q_pe, ws,
+                       input_norm_w=input_norm_w)
         return q_abs, q_pe
 
     def decode_attn(self, q_abs, q_pe, kv_cache, block_table, context_lens, max_context_len,

@@ -163,6 +163,16 @@ int mla_clear_device_flag(void* ws, void* stream);
 int mla_rope_cos_sin(const int32_t* positions, int n, int qk_rope, double theta,
                      float* cos_out, float* sin_out, void* stream);
 
+/* The same tables from a precomputed frequency table: angle_i = pos *
+ * inv_freq[i], evaluated in fp64 and rounded once to fp32. This is how a YaRN
+ * (or any other) frequency scaling enters ("Struct MlaWeights", yarn_inv_freq:
+ * a precomputed [rotary_dim/2] fp32 table; NULL there selects the plain theta
+ * computation, mla_rope_cos_sin here). YaRN's magnitude correction enters the
+ * score scale, mla_config.softmax_scale ("struct Mla", scale).
+ * inv_freq device [qk_rope/2] fp32; positions, cos_out, sin_out as above. */
+int mla_rope_cos_sin_inv_freq(const int32_t* positions, int n, int qk_rope, const float* inv_freq,
+                              float* cos_out, float* sin_out, void* stream);
+
 /* ---- decode ----------------------------------------------------------------- */
 
 /* The decode front-fold ("MLA Decode QKV Kernel API Reference",
@@ -180,7 +190,10 @@ int mla_rope_cos_sin(const int32_t* positions, int n, int qk_rope, double theta,
  *             MLA_FLAG_BAD_SLOT and skips. Slots must be distinct.
  * q_abs       device [n, H, r_kv] act dtype (output)
  * q_pe        device [n, H, d_r] act dtype (output)
- * input_norm_w must be NULL (a folded input RMSNorm is not implemented).
+ * input_norm_w device [D] fp32, or NULL. When given, the layer's input
+ *             RMSNorm is applied first: x <- x * rsqrt(mean(x^2) + norm_eps) *
+ *             input_norm_w, rounded to the activation dtype ("MLA Decode QKV
+ *             Kernel API Reference", input_norm_w: folded into the hidden load).
  * ws          device workspace (mla_workspace_bytes with max_tokens >= n). */
 int mla_decode_qkv(mla_handle* h, const void* hidden, int n, const float* cos,
                    const float* sin, void* kv_cache, int n_blocks,

@@ -79,8 +79,13 @@ def compact(inp, seqs, shape):
 class DecodeCase:
     """A decode step on the GPU and its inputs, for one workload."""
 
-    def __init__(self, workload, batch=None, ctx=None, row_layout=ref.LATENT_FIRST, device="cuda"):
+    def __init__(self, workload, batch=None, ctx=None, row_layout=ref.LATENT_FIRST, device="cuda",
+                 input_norm_w=None, inv_freq=None):
+        """input_norm_w [hidden] / inv_freq [qk_rope/2]: optional fp32 numpy arrays for
+        this step's input RMSNorm and RoPE frequency table (both sides get the same values)."""
         ensure_built()
+        self.input_norm_w = None if input_norm_w is None else np.asarray(input_norm_w, np.float32)
+        self.inv_freq = None if inv_freq is None else np.asarray(inv_freq, np.float32)
         self.w = workload
         self.shape = s = workload.shape
         self.row_layout = row_layout
@@ -95,7 +100,9 @@ class DecodeCase:
             self._fill_by_projection()
         self.hidden = to_dev(inp.hidden, self.act, device)
         self.positions = torch.from_numpy(inp.positions).to(device)
-        self.cos, self.sin = self.layer.rope(self.positions)
+        self.g_in = None if self.input_norm_w is None else torch.from_numpy(self.input_norm_w).to(device)
+        f = None if self.inv_freq is None else torch.from_numpy(self.inv_freq).to(device)
+        self.cos, self.sin = self.layer.rope(self.positions, f)
         self.slot = torch.from_numpy(inp.slot_mapping).to(device)
         self.table = torch.from_numpy(inp.block_table).to(device)
         self.ctx = torch.from_numpy(inp.context_lens).to(device)
@@ -115,7 +122,8 @@ class DecodeCase:
 
     def run(self):
         s = self.shape
-        self.q_abs, self.q_pe = self.layer.decode_qkv(self.hidden, self.cos, self.sin, self.cache, self.slot)
+        self.q_abs, self.q_pe = self.layer.decode_qkv(self.hidden, self.cos, self.sin, self.cache, self.slot,
+                                                      input_norm_w=self.g_in)
         n = self.hidden.shape[0]
         self.head_out = torch.empty((n, s.n_heads, s.v_dim), dtype=self.act, device=self.device)
         self.out = self.layer.decode_attn(self.q_abs, self.q_pe, self.cache, self.table, self.ctx,
@@ -140,9 +148,9 @@ class DecodeCase:
         if inp.fill_hidden is not None:
             cache = ref.fill_cache_by_projection(s, W, cache, [inp.fill_hidden[b] for b in seqs],
                                                  fill_slots, self.row_layout)
-        cos, sin = ref.rope_cos_sin(inp.positions[seqs], s.qk_rope, s.rope_theta)
+        cos, sin = ref.rope_cos_sin(inp.positions[seqs], s.qk_rope, s.rope_theta, inv_freq=self.inv_freq)
         q_abs, q_pe, new_cache = ref.decode_qkv(s, W, inp.hidden[seqs], cos, sin, cache, slots,
-                                                self.row_layout)
+                                                self.row_layout, input_norm_w=self.input_norm_w)
         out, head_out = ref.decode_attn(s, W, q_abs, q_pe, new_cache, table,
                                         inp.context_lens[seqs], self.row_layout)
         return dict(q_abs=q_abs, q_pe=q_pe, cache=new_cache, out=out, head_out=head_out,

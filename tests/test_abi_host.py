@@ -112,6 +112,9 @@ def test_calls_reject_null_handle_and_bad_sizes(lib):
     assert lib.mla_rope_cos_sin(P, -1, 16, 10000.0, P, P, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_rope_cos_sin(P, 4, 16, -1.0, P, P, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_rope_cos_sin(None, 0, 16, 10000.0, None, None, None) == mla.MLA_OK  # empty
+    assert lib.mla_rope_cos_sin_inv_freq(P, 4, 15, P, P, P, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_rope_cos_sin_inv_freq(P, 4, 16, None, P, P, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_rope_cos_sin_inv_freq(None, 0, 16, None, None, None, None) == mla.MLA_OK  # empty
     assert lib.mla_workspace_init(None, 1024, None) == mla.MLA_ERR_INVALID_ARG
     v = ctypes.c_int()
     assert lib.mla_read_device_flag(None, ctypes.byref(v), None) == mla.MLA_ERR_INVALID_ARG
