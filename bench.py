@@ -506,8 +506,8 @@ def workload_config(w: wl.Workload, world: int, context_lens=None) -> dict:
     s = w.shape
     l2 = "flushed before each timed step (256 MiB write, outside the events)"
     if w.mode == "prefill":
-        return {"workload": w.name, "seq_len": w.seq_len, "batch": 1, "heads": s.n_heads, "hidden": s.hidden,
-                "l2": l2, "parallelism": f"replicas x{world}"}
+        return {"workload": w.name, "seq_len": w.seq_len, "batch": 1, "weights": s.weight_dtype, "heads": s.n_heads,
+                "hidden": s.hidden, "l2": l2, "parallelism": f"replicas x{world}"}
     if context_lens is None:
         context_lens = wl._context_lens(w, np.random.default_rng(w.seed + 100))   # as make_decode_inputs draws them
     return {"workload": w.name, "batch": w.batch, "context": [int(context_lens.min()), int(context_lens.max())],

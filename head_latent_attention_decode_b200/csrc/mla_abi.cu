@@ -107,9 +107,10 @@ static WeightLayout make_layout(const mla_config* c) {
 // scratch share one region (calls on one workspace are stream-ordered).
 struct WsLayout {
   size_t Y1, qn, Q, part_o, part_ml, o_lat, head, xn;         // decode
-  size_t pY1, pqn, pQ, pcn, pkpe, pKV, phead;                  // prefill
+  size_t pY1, pqn, pQ, pcn, pkpe, pKV, phead, pDQ;             // prefill
   size_t tc;                                                   // tensor-core path scratch
-  size_t total;
+  size_t dec_total;                                            // what the decode calls need
+  size_t total;                                                // what every call needs
   int splits;
 };
 
@@ -137,6 +138,7 @@ static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
   W.xn = put((size_t)n * c->hidden * a);
   W.tc = put(tc_decode_ws_bytes(h, n, max_ctx));
   const size_t dec_end = off;
+  W.dec_total = dec_end;
   off = 256;
   W.pY1 = put((size_t)n * L.N1 * 4);
   W.pqn = put((size_t)n * (c->q_lora_rank ? c->q_lora_rank : 1) * a);
@@ -145,6 +147,7 @@ static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
   W.pkpe = put((size_t)n * dr * a);
   W.pKV = put((size_t)n * L.Hkv * a);
   W.phead = put((size_t)n * H * dv * a);
+  W.pDQ = put(tc_prefill_dequant_bytes(h));   // FP8 weights: one dequantised weight at a time
   W.total = dec_end > off ? dec_end : off;
   return W;
 }
@@ -215,6 +218,13 @@ static int acode(const mla_handle* h) { return h->cfg.act_dtype == MLA_F32 ? 0 :
 // ---------------------------------------------------------------------------
 // entry points
 // ---------------------------------------------------------------------------
+// The decode calls' own requirement (mla_workspace_bytes also covers prefill,
+// whose FP8 weight dequantisation buffer decode never touches).
+size_t mla_decode_workspace_bytes_internal(const mla_handle* h, int n) {
+  if (!h || n < 1) return 0;
+  return make_ws(h, n, 1).dec_total;
+}
+
 extern "C" {
 
 const char* mla_strerror(int s) {
@@ -320,6 +330,7 @@ size_t mla_workspace_bytes(const mla_handle* h, int max_tokens, int max_context_
   return make_ws(h, max_tokens, max_context_len).total;
 }
 
+
 int mla_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < 256) return MLA_ERR_INVALID_ARG;
   if (cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
@@ -374,7 +385,7 @@ int mla_decode_qkv(mla_handle* h, const void* hidden, int n, const float* cos, c
     return MLA_ERR_INVALID_ARG;
   const mla_config* c = &h->cfg;
   const WsLayout W = make_ws(h, n, 1);
-  if (ws_bytes < W.total) return MLA_ERR_WORKSPACE;
+  if (ws_bytes < W.dec_total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   char* wsb = (char*)ws;
   int* flag = (int*)wsb;
@@ -441,7 +452,7 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
   if (max_context_len < 1 || max_blocks_per_seq < 1) return MLA_ERR_INVALID_ARG;
   const mla_config* c = &h->cfg;
   const WsLayout W = make_ws(h, n, max_context_len);
-  if (ws_bytes < W.total) return MLA_ERR_WORKSPACE;
+  if (ws_bytes < W.dec_total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   char* wsb = (char*)ws;
   int* flag = (int*)wsb;
@@ -564,7 +575,7 @@ int mla_decode_step_host(mla_handle* h, const void* hidden_host, const int32_t* 
   if (max_blocks_per_seq < 1 || max_context_len < 1 || !(rope_theta > 0.0)) return MLA_ERR_INVALID_ARG;
   const StepStage P = make_stage(h, n, max_blocks_per_seq);
   if (stage_bytes < P.total) return MLA_ERR_WORKSPACE;
-  if (ws_bytes < make_ws(h, n, max_context_len).total) return MLA_ERR_WORKSPACE;
+  if (ws_bytes < make_ws(h, n, max_context_len).dec_total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   // pack the int32 inputs into the handle's page-locked buffer: one transfer
   if (h->pack_done && cudaEventSynchronize(h->pack_done) != cudaSuccess) return cuda_fail();
@@ -658,7 +669,7 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos, cons
   void* head = head_out ? head_out : (void*)(wsb + W.phead);
   if (tc_prefill_supported(h, S)) {
     const int r = tc_prefill(h, hidden, S, cos, sin, out, head, kv_cache, n_blocks, slot_mapping, wsb,
-                             W.pY1, W.pqn, W.pQ, W.pcn, W.pkpe, W.pKV, s);
+                             W.pY1, W.pqn, W.pQ, W.pcn, W.pkpe, W.pKV, W.pDQ, s);
     return r != MLA_OK ? r : cuda_status();
   }
   float* Y1 = (float*)(wsb + W.pY1);

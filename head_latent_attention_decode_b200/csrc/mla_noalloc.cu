@@ -16,6 +16,10 @@
 
 #include "../../include/mla.h"
 
+// Workspace bytes the decode front-fold needs for n tokens, without the
+// prefill-only buffers (mla_abi.cu).
+size_t mla_decode_workspace_bytes_internal(const mla_handle* h, int n);
+
 // The scratch itself. In host code this name is only a host-side stand-in for
 // the device symbol: the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
@@ -43,7 +47,7 @@ extern "C" int mla_decode_qkv_noalloc(mla_handle* h, const void* hidden, int n, 
                                       const int32_t* slot_mapping, void* q_abs, void* q_pe, void* stream) {
   if (!h || n < 0) return MLA_ERR_INVALID_ARG;
   if (n == 0) return MLA_OK;
-  const size_t need = mla_workspace_bytes(h, n, 1);
+  const size_t need = mla_decode_workspace_bytes_internal(h, n);
   if (need == 0) return MLA_ERR_INVALID_ARG;
   if (need > (size_t)MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;   // batch too large for the array
   void* ws = nullptr;

@@ -499,6 +499,38 @@ __global__ void rope_table_freq_kernel(const int* pos, int n, int d_r, const flo
   }
 }
 
+// FP8-E4M3 weight codes with 128 x 128 block scales to bf16, for the prefill
+// GEMMs: out[n][k] = bf16(e4m3(code[n][k]) * scale[n / 128][k / 128]) over a
+// K-major [N, K] matrix whose scales are [ceil(N/128)][ceil(K/128)] ("Struct
+// MlaWeights", wq_a_fp8: dequantised in fp32 before the MAC with bf16
+// activations). 16 codes per thread; K a multiple of 16.
+__global__ void dequant_fp8_bf16_kernel(const uint8_t* codes, const float* scales, long long N, long long K,
+                                        bf16* out) {
+  const long long kb = (K + 127) / 128;
+  const long long total = N * (K / 16);
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long n = idx / (K / 16), k0 = (idx % (K / 16)) * 16;
+    const float sc = scales[(n / 128) * kb + k0 / 128];
+    const uint4 c = *reinterpret_cast<const uint4*>(codes + n * K + k0);
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const float lo = e4m3_to_f32((uint8_t)(w[j] >> (16 * b))) * sc;
+        const float hi = e4m3_to_f32((uint8_t)(w[j] >> (16 * b + 8))) * sc;
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        o[2 * j + b] = *reinterpret_cast<uint32_t*>(&v);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + n * K + k0);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 // The layer's input RMSNorm, one CTA per token: xn = x * rsqrt(mean(x^2) + eps)
 // * gamma in the activation dtype ("MLA Decode QKV Kernel API Reference",
 // input_norm_w: the input RMSNorm folded into the hidden load).

@@ -376,6 +376,7 @@ static inline int tc_init(mla_handle* h) {
   T.enabled = 0;
   T.attn = 0;
   T.fp8 = 0;
+  T.pf8 = 0;
   int dev = 0, major = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -395,6 +396,10 @@ static inline int tc_init(mla_handle* h) {
     st |= make_map(&T.a8_Wuv, b + L.Wuv, rkv, dv, H, rkv, dv * rkv, 128, 0, true);
     st |= make_map(&T.a8_Wo, b + L.Wo, H * dv, D, 1, H * dv, H * dv * D, 128, 0, true);
     if (st == MLA_OK) T.fp8 = 1;
+    // prefill: the same shape limits as the bf16 tensor-core prefill
+    if (c.hidden % 64 == 0 && c.kv_lora_rank % 64 == 0 && c.qk_nope % 64 == 0 && c.q_lora_rank % 64 == 0 &&
+        ((long long)c.n_heads * c.v_dim) % 64 == 0)
+      T.pf8 = 1;
     return MLA_OK;
   }
   if (major != 10 || c.act_dtype != MLA_BF16 || c.weight_dtype != MLA_BF16) return MLA_OK;
@@ -429,7 +434,36 @@ static inline bool tc_decode_attn_supported(const mla_handle* h, int n, int) {
 }
 
 static inline bool tc_attention_supported(const mla_handle* h) { return h->tc.attn != 0; }
-static inline bool tc_prefill_supported(const mla_handle* h, int) { return h->tc.enabled; }
+static inline bool tc_prefill_supported(const mla_handle* h, int) { return h->tc.enabled || h->tc.pf8; }
+
+// Bytes of the bf16 buffer FP8 handles dequantise each prefill weight into (the largest of them).
+static inline size_t tc_prefill_dequant_bytes(const mla_handle* h) {
+  if (!h->tc.pf8) return 0;
+  const WeightLayout& L = h->L;
+  const mla_config& c = h->cfg;
+  long long m = (long long)L.N1 * c.hidden;
+  if (c.q_lora_rank) m = m > (long long)L.Hq * c.q_lora_rank ? m : (long long)L.Hq * c.q_lora_rank;
+  m = m > (long long)L.Hkv * c.kv_lora_rank ? m : (long long)L.Hkv * c.kv_lora_rank;
+  m = m > (long long)c.hidden * c.n_heads * c.v_dim ? m : (long long)c.hidden * c.n_heads * c.v_dim;
+  return (size_t)m * 2;
+}
+
+// The B-operand map (256-row boxes) of prefill weight [N, K] starting at row
+// `row0`: the resident bf16 weights, or, for FP8 handles, the weight just
+// dequantised into `dq` (rows [0, N) of it; launched here, on `s`).
+static inline int prefill_weight_map(const mla_handle* h, CUtensorMap* m, const CUtensorMap& bf16_map,
+                                     size_t codes_off, size_t scales_off, long long N, long long K, long long row0,
+                                     long long rows, char* dq, bool dequant, cudaStream_t s) {
+  if (!h->tc.pf8) { *m = bf16_map; return MLA_OK; }
+  if (dequant) {
+    const long long total = N * (K / 16);
+    const int blocks = (int)(cdiv(total, 256) > 8 * 148 ? 8 * 148 : cdiv(total, 256));
+    dequant_fp8_bf16_kernel<<<blocks, 256, 0, s>>>((const uint8_t*)(h->base + codes_off),
+                                                   (const float*)(h->base + scales_off), N, K, (bf16*)dq);
+    mla_count_launch(1);
+  }
+  return make_map2(m, dq + (size_t)row0 * K * 2, K, rows, K, 256);
+}
 
 enum WSel { W_1, W_QB, W_UK, W_UV, W_O };
 
@@ -684,7 +718,7 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
 static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, const float* cos, const float* sin,
                              void* out, void* head, void* kv_cache, int n_blocks, const int32_t* slot_mapping,
                              char* ws, size_t pY1, size_t pqn, size_t pQ, size_t pcn, size_t pkpe, size_t pKV,
-                             cudaStream_t s) {
+                             size_t pDQ, cudaStream_t s) {
   const mla_config& c = h->cfg;
   const WeightLayout& L = h->L;
   const TcState& T = h->tc;
@@ -692,6 +726,10 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
   const int H = c.n_heads, dn = c.qk_nope, dr = c.qk_rope, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
   const int rq = c.q_lora_rank;
   int st;
+  // FP8 handles dequantise each weight into `dq` just before its GEMM; that GEMM then
+  // must not load its weights ahead of its dependency wait (static_op 0)
+  char* dq = T.pf8 ? ws + pDQ : nullptr;
+  const int sop = T.pf8 ? 0 : 2;
   CUtensorMap mx;
   if ((st = make_map2(&mx, hidden, D, S, D, 128)) != MLA_OK) return st;
   float* Y1 = (float*)(ws + pY1);
@@ -699,14 +737,23 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
   FrontFoldArgs f{};
   if (rq) {
     GemmArgs g = gemm_args(S, L.N1, D, 1, EPI_F32_N, Y1, L.N1, 0, flag);
-    if ((st = launch_gemm(mx, T.b_W1, g, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+    CUtensorMap bw;
+    if ((st = prefill_weight_map(h, &bw, T.b_W1, L.W1, L.sW1, L.N1, D, 0, L.N1, dq, true, s)) != MLA_OK) return st;
+    g.static_op = sop;
+    if ((st = launch_gemm(mx, bw, g, 256, 1, T.num_sms, s)) != MLA_OK) return st;
     f.Y = Y1; f.ldy = L.N1; f.kv0 = L.Nq1;
   } else {
     GemmArgs gq = gemm_args(S, L.Hq, D, 1, EPI_QROPE_N, Q, L.Hq, 0, flag);
     gq.cos = cos; gq.sin = sin; gq.H = H; gq.dn = dn; gq.dr = dr;
-    if ((st = launch_gemm(mx, T.b_W1q, gq, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+    CUtensorMap bq, bk;
+    if ((st = prefill_weight_map(h, &bq, T.b_W1q, L.W1, L.sW1, L.N1, D, 0, L.Nq1, dq, true, s)) != MLA_OK) return st;
+    if ((st = prefill_weight_map(h, &bk, T.b_W1kv, L.W1, L.sW1, L.N1, D, L.Nq1, L.R, dq, false, s)) != MLA_OK)
+      return st;
+    gq.static_op = sop;
+    if ((st = launch_gemm(mx, bq, gq, 256, 1, T.num_sms, s)) != MLA_OK) return st;
     GemmArgs gk = gemm_args(S, L.R, D, 1, EPI_F32_N, Y1, L.R, 0, flag);
-    if ((st = launch_gemm(mx, T.b_W1kv, gk, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+    gk.static_op = sop;
+    if ((st = launch_gemm(mx, bk, gk, 256, 1, T.num_sms, s)) != MLA_OK) return st;
     f.Y = Y1; f.ldy = L.R; f.kv0 = 0;
   }
   f.r_q = rq; f.r_kv = rkv; f.d_r = dr;
@@ -724,13 +771,20 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
     if ((st = make_map2(&mq, ws + pqn, rq, S, rq, 128)) != MLA_OK) return st;
     GemmArgs g2 = gemm_args(S, L.Hq, rq, 1, EPI_QROPE_N, Q, L.Hq, 0, flag);
     g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr;
-    if ((st = launch_gemm(mq, T.b_Wqb, g2, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+    CUtensorMap bw;
+    if ((st = prefill_weight_map(h, &bw, T.b_Wqb, L.Wqb, L.sWqb, L.Hq, rq, 0, L.Hq, dq, true, s)) != MLA_OK) return st;
+    g2.static_op = sop;
+    if ((st = launch_gemm(mq, bw, g2, 256, 1, T.num_sms, s)) != MLA_OK) return st;
   }
   CUtensorMap mc;
   if ((st = make_map2(&mc, ws + pcn, rkv, S, rkv, 128)) != MLA_OK) return st;
   bf16* KV = (bf16*)(ws + pKV);
   GemmArgs g3 = gemm_args(S, L.Hkv, rkv, 1, EPI_BF16_N, KV, L.Hkv, 0, flag);
-  if ((st = launch_gemm(mc, T.b_Wkvb, g3, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+  CUtensorMap bkv;
+  if ((st = prefill_weight_map(h, &bkv, T.b_Wkvb, L.Wkvb, L.sWkvb, L.Hkv, rkv, 0, L.Hkv, dq, true, s)) != MLA_OK)
+    return st;
+  g3.static_op = sop;
+  if ((st = launch_gemm(mc, bkv, g3, 256, 1, T.num_sms, s)) != MLA_OK) return st;
   if (dn == 128 && dr == 64 && dv == 128) {
     CUtensorMap mq, mkv, mkpe;
     if ((st = make_map2(&mq, Q, L.Hq, S, L.Hq, 128)) != MLA_OK) return st;
@@ -766,5 +820,9 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
   CUtensorMap mh;
   if ((st = make_map2(&mh, head, (long long)H * dv, S, (long long)H * dv, 128)) != MLA_OK) return st;
   GemmArgs g5 = gemm_args(S, D, H * dv, 1, EPI_BF16_N, out, D, 0, flag);
-  return launch_gemm(mh, T.b_Wo, g5, 256, 1, T.num_sms, s);
+  CUtensorMap bo;
+  if ((st = prefill_weight_map(h, &bo, T.b_Wo, L.Wo, L.sWo, D, (long long)H * dv, 0, D, dq, true, s)) != MLA_OK)
+    return st;
+  g5.static_op = sop;
+  return launch_gemm(mh, bo, g5, 256, 1, T.num_sms, s);
 }

@@ -8,6 +8,7 @@ struct TcState {
   int enabled;       // bf16 activations with bf16 weights on an sm_100 device (all tcgen05 GEMMs)
   int attn;          // bf16 activations on an sm_100 device (tcgen05 attention, any weight dtype)
   int fp8;           // FP8 weights with bf16 activations: tcgen05 decode GEMMs on decoded FP8 tiles
+  int pf8;           // FP8 weights, prefill on the bf16 tcgen05 path after a per-call dequantisation
   int num_sms;
   // weights as the A operand (decode, swap-AB): 128-row boxes
   CUtensorMap a_W1, a_Wqb, a_Wuk, a_Wuv, a_Wo;

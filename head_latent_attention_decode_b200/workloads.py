@@ -103,6 +103,10 @@ WORKLOADS = {
         "v3_prefill_bf16", V3, "prefill", batch=1, ctx_lo=0, ctx_hi=0, cache_fill="none",
         seed=4, seq_len=8192, description="DeepSeek-V3-shaped MLA prefill bf16, seq 8192 "
         "causal, expanded K/V"),
+    "v3_prefill_fp8": Workload(
+        "v3_prefill_fp8", V3_FP8, "prefill", batch=1, ctx_lo=0, ctx_hi=0, cache_fill="none",
+        seed=6, seq_len=8192, description="DeepSeek-V3-shaped MLA prefill, FP8-E4M3 weights with "
+        "128x128 fp32 block scales, bf16 activations, seq 8192 causal, expanded K/V"),
 }
 
 

@@ -142,7 +142,9 @@ void mla_destroy(mla_handle* h);
 
 /* Bytes of device workspace the calls below need for up to `max_tokens`
  * decode tokens (or prefill sequence length) and contexts of up to
- * `max_context_len` rows. */
+ * `max_context_len` rows. For FP8 weights this includes one bf16 buffer of
+ * the largest weight, into which mla_prefill dequantises each weight in turn
+ * (the decode calls never use it and accept a workspace without it). */
 size_t mla_workspace_bytes(const mla_handle* h, int max_tokens, int max_context_len);
 
 /* Zero the workspace (device flag and internal counters). Call once on a new
@@ -236,9 +238,9 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe,
  * MLA_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
  * process exits. The first call on a device looks up that array's address
  * (cudaGetSymbolAddress) with the device current; make that first call before
- * any stream capture. Returns MLA_ERR_WORKSPACE when
- * mla_workspace_bytes(h, n, 1) exceeds the array (for the DeepSeek-V3 shape
- * that allows about 64 tokens per call). All calls share the one array, whose
+ * any stream capture. Returns MLA_ERR_WORKSPACE when the front-fold's
+ * workspace for n tokens exceeds the array (for the DeepSeek-V3 shape that
+ * allows about 64 tokens per call). All calls share the one array, whose
  * contents persist between calls: each call clears the device flag it holds
  * (so the flag is not readable here), and calls that overlap on the GPU, on
  * any streams, race. Calls no cudaMalloc, cudaFree or allocating routine. */

@@ -17,6 +17,7 @@ pytestmark = pytest.mark.gpu
 
 TINY_PREFILL = dataclasses.replace(wl.WORKLOADS["v3_prefill_bf16"], shape=wl.TINY, seed=9)
 V2LITE_PREFILL = dataclasses.replace(wl.WORKLOADS["v3_prefill_bf16"], shape=wl.V2LITE, seed=10)
+V3_FP8_PREFILL = dataclasses.replace(wl.WORKLOADS["v3_prefill_bf16"], shape=wl.WORKLOADS["v3_fp8"].shape, seed=12)
 
 
 def run_prefill(workload, S, rows=None, with_cache=False):
@@ -74,6 +75,13 @@ def test_v2lite_bf16_prefill_tile_edges(S):
 
 def test_v3_bf16_prefill_small():
     run_prefill(wl.WORKLOADS["v3_prefill_bf16"], S=300, with_cache=True)
+
+
+@pytest.mark.parametrize("S", [129, 300])
+def test_v3_fp8_weights_prefill(S):
+    """FP8-E4M3 weights with 128 x 128 block scales on the tensor-core prefill:
+    each weight dequantised into the workspace just before its GEMM."""
+    run_prefill(V3_FP8_PREFILL, S=S, with_cache=True)
 
 
 def test_v3_bf16_prefill_full_sampled():
