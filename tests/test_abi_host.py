@@ -123,3 +123,16 @@ def test_calls_reject_null_handle_and_bad_sizes(lib):
 
 def test_launch_counter_starts_at_zero_without_gpu_work(lib):
     assert mla.mla_kernel_launch_count() == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No silent fallback: without the built library every entry point raises."""
+    from head_latent_attention_decode_b200.layer import MlaLayer
+    monkeypatch.setattr(mla, "LIB_PATH", str(tmp_path / "libmla_b200.so"))
+    monkeypatch.setattr(mla, "_lib", None)
+    with pytest.raises(ImportError):
+        mla.lib()
+    with pytest.raises(ImportError):
+        mla.mla_weights_bytes(mla.make_config(wl.TINY))
+    with pytest.raises(ImportError):
+        MlaLayer(wl.TINY, wl.make_weights(wl.TINY, 0), device="cpu")
