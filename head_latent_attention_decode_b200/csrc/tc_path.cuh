@@ -336,16 +336,20 @@ using namespace mla;
 using namespace mla::tc;
 
 struct TcDecodeWs {
-  size_t Yp, qn, q_nope, wo_part, bf16c, total;
+  size_t Yp, qn, q_nope, wo_part, bf16c, dq, total;
   int s1, s5;
+  bool deq;   // FP8 weights beyond the FP8 GEMM's 128 tokens: dequantise each weight into dq, bf16 GEMMs
 };
+
+static inline size_t tc_prefill_dequant_bytes(const mla_handle* h);
 
 static TcDecodeWs tc_decode_ws(const mla_handle* h, long long n) {
   TcDecodeWs w{};
   const mla_config& c = h->cfg;
   const WeightLayout& L = h->L;
   const int sms = h->tc.num_sms > 0 ? h->tc.num_sms : 148;
-  const int ku = h->tc.fp8 ? 128 : 64;   // K block of the GEMM kernel in use
+  w.deq = h->tc.fp8 && n > 128;
+  const int ku = h->tc.fp8 && !w.deq ? 128 : 64;   // K block of the GEMM kernel in use
   w.s1 = decode_splits_for((int)cdiv(L.N1, 128), (int)cdiv(c.hidden, ku), sms);
   w.s5 = decode_splits_for((int)cdiv(c.hidden, 128), (int)cdiv((long long)c.n_heads * c.v_dim, ku), sms);
   size_t off = 0;
@@ -354,7 +358,8 @@ static TcDecodeWs tc_decode_ws(const mla_handle* h, long long n) {
   w.qn = put((size_t)n * (c.q_lora_rank ? c.q_lora_rank : 8) * 2);
   w.q_nope = put((size_t)n * c.n_heads * c.qk_nope * 2);
   w.wo_part = put((size_t)w.s5 * n * c.hidden * 4);
-  if (h->tc.fp8) {   // f16 copy of the largest token operand of an FP8 GEMM
+  if (w.deq) w.dq = put(tc_prefill_dequant_bytes(h));   // one dequantised weight at a time
+  if (h->tc.fp8 && !w.deq) {   // f16 copy of the largest token operand of an FP8 GEMM
     long long e = c.hidden;
     if (c.q_lora_rank > e) e = c.q_lora_rank;
     if ((long long)c.n_heads * c.qk_nope > e) e = (long long)c.n_heads * c.qk_nope;
@@ -426,11 +431,17 @@ static inline int tc_init(mla_handle* h) {
   return MLA_OK;
 }
 
+// FP8 weights take the FP8 GEMMs up to 128 tokens and, up to 256, the bf16
+// GEMMs on weights dequantised per call (flattening the per-head W_UK / W_UV
+// scale blocks needs r_kv and d_v to be multiples of 128).
+static inline bool tc_decode_fp8_dequant_ok(const mla_handle* h) {
+  return h->tc.pf8 && h->cfg.v_dim % 128 == 0 && h->cfg.kv_lora_rank % 128 == 0;
+}
 static inline bool tc_decode_qkv_supported(const mla_handle* h, int n) {
-  return (h->tc.enabled && n <= 256) || (h->tc.fp8 && n <= 128);
+  return (h->tc.enabled && n <= 256) || (h->tc.fp8 && n <= 128) || (tc_decode_fp8_dequant_ok(h) && n <= 256);
 }
 static inline bool tc_decode_attn_supported(const mla_handle* h, int n, int) {
-  return (h->tc.enabled && n <= 256) || (h->tc.fp8 && n <= 128);
+  return (h->tc.enabled && n <= 256) || (h->tc.fp8 && n <= 128) || (tc_decode_fp8_dequant_ok(h) && n <= 256);
 }
 
 static inline bool tc_attention_supported(const mla_handle* h) { return h->tc.attn != 0; }
@@ -479,9 +490,10 @@ static BView bview2(const void* p, long long K, long long rows) { return BView{p
 
 // Weight GEMM of the decode path: bf16 weights on tc_gemm_kernel, FP8 weights
 // on tc_gemm_fp8_kernel (tokens converted to f16 into `f16buf` first) with the
-// matrix's block scales.
+// matrix's block scales, or, given `dq`, on tc_gemm_kernel after dequantising
+// the weight into it.
 static int wgemm(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int bn, int splits, void* f16buf,
-                 cudaStream_t s) {
+                 char* dq, cudaStream_t s) {
   const TcState& T = h->tc;
   CUtensorMap B;
   int st;
@@ -490,6 +502,37 @@ static int wgemm(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int b
     if ((st = make_map(&B, bv.p, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
     const CUtensorMap* A = w == W_1 ? &T.a_W1 : w == W_QB ? &T.a_Wqb : w == W_UK ? &T.a_Wuk : w == W_UV ? &T.a_Wuv : &T.a_Wo;
     return launch_gemm(*A, B, g, bn, splits, T.num_sms, s);
+  }
+  if (dq) {
+    // FP8 weights, more tokens than the FP8 GEMM takes: dequantise the weight to bf16
+    // [N, K] (per-head blocks stacked) and run the bf16 GEMM on it; the GEMM must not
+    // load the weight ahead of its dependency wait
+    const WeightLayout& L = h->L;
+    const mla_config& c = h->cfg;
+    const long long D = c.hidden, rq = c.q_lora_rank, dn = c.qk_nope, dv = c.v_dim, rkv = c.kv_lora_rank;
+    const long long H = c.n_heads;
+    size_t co, so;
+    long long N, K;
+    switch (w) {
+      case W_1: co = L.W1; so = L.sW1; N = L.N1; K = D; break;
+      case W_QB: co = L.Wqb; so = L.sWqb; N = L.Hq; K = rq; break;
+      case W_UK: co = L.Wuk; so = L.sWuk; N = H * rkv; K = dn; break;
+      case W_UV: co = L.Wuv; so = L.sWuv; N = H * dv; K = rkv; break;
+      default: co = L.Wo; so = L.sWo; N = D; K = H * dv; break;
+    }
+    const long long total = N * (K / 16);
+    const int blocks = (int)(cdiv(total, 256) > 8 * 148 ? 8 * 148 : cdiv(total, 256));
+    dequant_fp8_bf16_kernel<<<blocks, 256, 0, s>>>((const uint8_t*)(h->base + co), (const float*)(h->base + so), N,
+                                                   K, (bf16*)dq);
+    mla_count_launch(1);
+    CUtensorMap A;
+    if (w == W_UK) st = make_map(&A, dq, dn, rkv, H, dn * 2, rkv * dn * 2, 128, 0);
+    else if (w == W_UV) st = make_map(&A, dq, rkv, dv, H, rkv * 2, dv * rkv * 2, 128, 0);
+    else st = make_map2(&A, dq, K, N, K, 128);
+    if (st != MLA_OK) return st;
+    if ((st = make_map(&B, bv.p, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
+    g.static_op = 0;
+    return launch_gemm(A, B, g, bn, splits, T.num_sms, s);
   }
   if ((((uintptr_t)bv.p) & 15) || (bv.elems % 8)) return MLA_ERR_UNSUPPORTED;
   const long long n8 = bv.elems / 8;
@@ -538,8 +581,9 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   int st;
   // 1. Yp[split] = x @ W1 (swap-AB: A = W1 [N1, D], B = x [n, D])
   void* f16buf = tw + W.bf16c;
+  char* dq = W.deq ? tw + W.dq : nullptr;
   GemmArgs g = gemm_args(L.N1, n, D, 1, EPI_F32_T, tw + W.Yp, L.N1, 0, flag);
-  if ((st = wgemm(h, W_1, bview2(hidden, D, n), g, bn, W.s1, f16buf, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_1, bview2(hidden, D, n), g, bn, W.s1, f16buf, dq, s)) != MLA_OK) return st;
   // 2. split sum, norms, RoPE, scatter (and, without q_lora, q_nope / q_pe)
   FrontFoldTcArgs f{};
   f.Yp = (const float*)(tw + W.Yp); f.split_stride = (long long)n * L.N1; f.splits = W.s1; f.N1 = L.N1;
@@ -559,13 +603,13 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
 
     GemmArgs g2 = gemm_args(L.Hq, n, rq, 1, EPI_QROPE_T, tw + W.q_nope, 0, 0, flag);
     g2.out2 = q_pe; g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr;
-    if ((st = wgemm(h, W_QB, bview2(tw + W.qn, rq, n), g2, bn, 1, f16buf, s)) != MLA_OK) return st;
+    if ((st = wgemm(h, W_QB, bview2(tw + W.qn, rq, n), g2, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
   }
   // 4. q_abs[h] = q_nope[h] @ W_UK[h]  (batched over heads: A = Wuk[h] [r_kv, d_n], B = q_nope[:, h, :])
   const BView vn{tw + W.q_nope, dn, H, n, dn, (long long)H * dn, (long long)n * H * dn, 1};
   GemmArgs g3 = gemm_args(rkv, n, dn, H, EPI_BF16_T, q_abs, (long long)H * rkv, rkv, flag);
   g3.b_rows_dim2 = 1;
-  return wgemm(h, W_UK, vn, g3, bn, 1, f16buf, s);
+  return wgemm(h, W_UK, vn, g3, bn, 1, f16buf, dq, s);
 }
 
 // Split-KV absorbed attention and the LSE merge of the splits -> o_lat (bf16).
@@ -701,13 +745,14 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   if (st != MLA_OK) return st;
   // 2. head_out[h] = o_lat[h] @ W_UV[h]  (A = Wuv[h] [d_v, r_kv], B = o_lat[:, h, :])
   void* f16buf = tw + W.bf16c;
+  char* dq = W.deq ? tw + W.dq : nullptr;
   const BView vo{o_lat, rkv, H, n, rkv, (long long)H * rkv, (long long)n * H * rkv, 1};
   GemmArgs g4 = gemm_args(dv, n, rkv, H, EPI_BF16_T, head, (long long)H * dv, dv, flag);
   g4.b_rows_dim2 = 1;
-  if ((st = wgemm(h, W_UV, vo, g4, bn, 1, f16buf, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_UV, vo, g4, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
   // 3. out = head_out @ wo  (swap-AB, K split, then reduce to bf16)
   GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
-  if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n), g5, bn, W.s5, f16buf, s)) != MLA_OK) return st;
+  if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n), g5, bn, W.s5, f16buf, dq, s)) != MLA_OK) return st;
   const long long cnt = (long long)n * D;
   launch_pdl(splitk_reduce_bf16_kernel, (unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s,
              (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);

@@ -106,6 +106,15 @@ def test_v3_bf16_full_sampled():
     check_case(case, seqs=seqs)
 
 
+@pytest.mark.parametrize("batch", [129, 200])
+def test_v3_fp8_more_tokens_than_the_fp8_gemm(batch):
+    """FP8 weights with 129..256 tokens per call: each weight dequantised to
+    bf16 in the workspace, then the bf16 tensor-core GEMMs (the FP8 GEMM takes
+    up to 128 tokens); sampled sequences against the oracle."""
+    case = DecodeCase(wl.WORKLOADS["v3_fp8"], batch=batch, ctx=(64, 300)).run()
+    check_case(case, seqs=[0, 77, batch - 1])
+
+
 def test_v3_fp8_full_sampled():
     case = DecodeCase(wl.WORKLOADS["v3_fp8"]).run()
     check_case(case, seqs=[0, 64, 127])
