@@ -8,7 +8,8 @@
 // 64-row cache tile:
 //   S_r = [q_abs | q_pe]_r . tile_r^T      (tcgen05, M 128 x N 64, K 256 / 320;
 //                                          the latent part of Q lives in TMEM)
-//   S   = S_0 + S_1                        (the partials swap through DSMEM)
+//   S   = S_0 + S_1                        (the partials swap through DSMEM in f16,
+//                                          into two alternating buffers)
 //   online softmax, one thread per head (nothing to reduce across threads),
 //   lazy rescale of the TMEM accumulator when the max grows by more than 2^8;
 //   P (bf16) is written back into TMEM over S
@@ -55,9 +56,9 @@ struct AttnSmem {
   static constexpr int STAGE = 5 * 8192;        // 4 latent + 1 rope slot of [64 rows x 64 cols] bf16
   static constexpr int TILE_OFF = 0;
   static constexpr int QR_OFF = ATT_NST * STAGE;  // q_pe [128 x 64] bf16 (CTA 0)
-  static constexpr int X_OFF = QR_OFF + 16384;    // [128 x 64] fp32, the peer's partial S
-  static constexpr int STG_OFF = X_OFF + 32768;   // [128 x 64] fp32, our partial on its way out
-  static constexpr int BAR_OFF = STG_OFF + 32768;
+  static constexpr int X_OFF = QR_OFF + 16384;    // 2 x [128 x 64] f16, the peer's partial S (double-buffered)
+  static constexpr int STG_OFF = X_OFF + 32768;   // [128 x 64] f16, our partial on its way out
+  static constexpr int BAR_OFF = STG_OFF + 16384;
   static constexpr int SIZE = 1024 + BAR_OFF + 256;
 };
 // TMEM columns: Q latent [0,128) (bf16 pairs), S/P buffers [128,192) [192,256), O [256,512)
@@ -90,7 +91,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   const uint32_t p_full_b = s_full_b + 16;             // [2]
   const uint32_t sp_empty_b = p_full_b + 16;           // [2] S/P buffer free (P.V done)
   const uint32_t q_ready = sp_empty_b + 16, qr_full = q_ready + 8, o_done = qr_full + 8;
-  const uint32_t x_full_b = o_done + 8, x_free_b = x_full_b + 16, fin = x_free_b + 16;   // x_full, x_free
+  const uint32_t x_full_b = o_done + 8, x_free_b = x_full_b + 16, fin = x_free_b + 16;   // x_full[2], x_free[2]
   const uint32_t s_read_b = fin + 8;   // [2] the sender has read S(t) out of TMEM
   uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 192);
   volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 196);
@@ -128,8 +129,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     mbar_init(q_ready, 128);
     mbar_init(qr_full, 1);
     mbar_init(o_done, 1);
-    mbar_init(x_full_b, 1);
-    mbar_init(x_free_b, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(x_full_b + 8 * i, 1);
+      mbar_init(x_free_b + 8 * i, 4);
+    }
     for (int i = 0; i < 2; ++i) mbar_init(s_read_b + 8 * i, 128);
     mbar_init(fin, 1);
     *abort_word = 0;
@@ -255,7 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     const bool issuer = (warp == 6 && lane == 0);
     const uint32_t peer_x = mapa_shared(x_s, peer), peer_x_full = mapa_shared(x_full_b, peer);
     const uint32_t stg_s = sbase + SM::STG_OFF;
-    float4* stg_row = (float4*)(smem + SM::STG_OFF + h * 256);
+    uint4* stg_row = (uint4*)(smem + SM::STG_OFF + h * 128);
     for (int k = 0; k < T; ++k) {
       const int kb = k & 1;
       if (!mbar_wait_warp(s_full_b + 8 * kb, (k >> 1) & 1, abort_word, a.flag)) break;
@@ -272,17 +275,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       if (trs) a.trace[k * 16 + 13] = global_timer_ns();
       if (issuer) bulk_wait_read_all();                  // the previous copy has left the staging buffer
       named_bar_sync(2, 128);
+      // the partial goes out in f16 (half the distributed-shared-memory bytes of fp32; the
+      // partial scores stay far inside f16's range and its 11-bit significand costs the
+      // scores ~1e-3 relative, well inside the output tolerance)
 #pragma unroll
-      for (int c = 0; c < 16; ++c)   // chunk c of row h at slot c ^ (h & 15): no bank conflicts
-        stg_row[c ^ (h & 15)] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      for (int c = 0; c < 8; ++c) {  // chunk c (8 values) of row h at slot c ^ (h & 7): no bank conflicts
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          __half2 hv = __floats2half2_rn(v[8 * c + 2 * j], v[8 * c + 2 * j + 1]);
+          w[j] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        stg_row[c ^ (h & 7)] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
       fence_proxy_async_smem();
       named_bar_sync(2, 128);
       if (issuer) {
-        // the peer has consumed what we sent for tile k - 1
-        bool ok = mbar_wait_cluster(x_free_b, (k & 1) ^ 1, abort_word, a.flag);
+        // the peer has consumed what we sent for tile k - 2 into the same buffer
+        const int xb = k & 1;
+        bool ok = mbar_wait_cluster(x_free_b + 8 * xb, ((k >> 1) & 1) ^ 1, abort_word, a.flag);
         if (trs) a.trace[k * 16 + 14] = global_timer_ns();
         if (ok) {
-          bulk_copy_to_peer(peer_x, stg_s, 32768, peer_x_full);
+          bulk_copy_to_peer(peer_x + xb * 16384, stg_s, 16384, peer_x_full + 8 * xb);
           bulk_commit_group();
         }
       }
@@ -320,8 +334,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       if (valid < 0) valid = 0;
       const bool tr = trace && h == 0 && t < 64;
       if (tr) trace[t * 16 + 0] = global_timer_ns();
-      if (h == 0) mbar_arrive_expect_tx(x_full_b, 32768);
-      if (!mbar_wait_warp(x_full_b, t & 1, abort_word, a.flag)) { ok = false; break; }
+      const int xb = t & 1;
+      if (h == 0) mbar_arrive_expect_tx(x_full_b + 8 * xb, 16384);
+      if (!mbar_wait_warp(x_full_b + 8 * xb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       if (tr) trace[t * 16 + 2] = global_timer_ns();
       if (!mbar_wait_warp(s_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       if (tr) trace[t * 16 + 6] = global_timer_ns();
@@ -332,15 +347,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
       for (int c = 0; c < 4; ++c) tmem_ld16(sp_addr + 16 * c, (uint32_t*)&v[16 * c]);
       tmem_ld_wait();
       if (tr) trace[t * 16 + 7] = global_timer_ns();
-      const float4* xloc = (const float4*)(smem + SM::X_OFF + h * 256);
+      const uint4* xloc = (const uint4*)(smem + SM::X_OFF + xb * 16384 + h * 128);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 x = xloc[c ^ (h & 15)];
-        v[4 * c] += x.x; v[4 * c + 1] += x.y; v[4 * c + 2] += x.z; v[4 * c + 3] += x.w;
+      for (int c = 0; c < 8; ++c) {
+        const uint4 x = xloc[c ^ (h & 7)];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+          v[8 * c + 2 * j] += f.x;
+          v[8 * c + 2 * j + 1] += f.y;
+        }
       }
       if (tr) trace[t * 16 + 11] = global_timer_ns();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote_relaxed(peer_x_free);
+      if (lane == 0) mbar_arrive_remote_relaxed(peer_x_free + 8 * xb);
       if (tr) trace[t * 16 + 3] = global_timer_ns();
       // online softmax in log2 units with a lazily moved reference max
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
