@@ -7,8 +7,9 @@
 //   rotary columns of the tiles t with t % 2 == r;
 //   S_r^T = tile_r . Q_r^T               M 128 rows x N NH heads, K 256 or 320
 //   S^T   = S_r^T + S_peer^T             each softmax thread sends its row (NH
-//                                        fp32) into the peer's shared memory with
-//                                        st.async, ahead of its own softmax
+//                                        values, in f16) into the peer's shared
+//                                        memory with st.async, ahead of its own
+//                                        softmax
 //   softmax down each head's column with a lazily moved reference max: the
 //   rows vote whether any score exceeds its head's reference by more than 2^8,
 //   and only then are the column maxima reduced (warp redux and a 4-warp
@@ -31,7 +32,7 @@ struct AttnPairSmem {
   // ring entries: [128 rows x 128 latent] bf16, 32 KB, laid out [16 row octets][2 k-blocks][8 rows][128 B]
   static constexpr int NPR = NH <= 16 ? 5 : 4;
   static constexpr int QKB = NH * 128;                   // one [NH x 64] bf16 k-block of Q or P^T
-  static constexpr int XB = 128 * NH * 4;                // one [128 x NH] fp32 partial S^T
+  static constexpr int XB = 128 * NH * 2;                // one [128 x NH] f16 partial S^T
   static constexpr int RING_OFF = 0;
   static constexpr int ROPE_OFF = NPR * 32768;           // [128 x 64] rotary block of the current tile
   static constexpr int Q_OFF = ROPE_OFF + 16384;         // this CTA's 4 latent k-blocks of Q, then q_pe
@@ -51,8 +52,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
   using SM = AttnPairSmem<NH>;
   griddep_wait();   // the inputs all come from the stream's earlier kernels
   constexpr int NPR = SM::NPR, QKB = SM::QKB;
-  constexpr int CPR = NH / 4;                  // 16-byte chunks per row of a partial
-  constexpr int XSH = NH == 16 ? 1 : 0;        // chunk swizzle: 8 consecutive rows cover all 32 banks
+  constexpr int CPR = NH / 8;                  // 16-byte chunks per row of an f16 partial
+  constexpr int XSH = NH == 16 ? 2 : 1;        // chunk swizzle: the rows of one 128-byte line cover all 32 banks
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -300,11 +301,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       // the peer has read what we sent for tile u - 2 out of this buffer
       if (!mbar_wait_cluster_warp(x_free_b + 8 * sb, ((u >> 1) & 1) ^ 1, abort_word, a.flag)) return false;
       if (tr0 && u < 64) trace[u * 32 + 7] = global_timer_ns();
-      const uint32_t dst = peer_x + sb * SM::XB + i * (NH * 4);
+      // the partial crosses in f16 (half the bytes; partial scores stay far inside its range)
+      const uint32_t dst = peer_x + sb * SM::XB + i * (NH * 2);
 #pragma unroll
-      for (int c = 0; c < CPR; ++c)
-        st_async_v4(dst + 16 * (c ^ xsw), nxt[4 * c], nxt[4 * c + 1], nxt[4 * c + 2], nxt[4 * c + 3],
-                    peer_x_full + 8 * sb);
+      for (int c = 0; c < CPR; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          __half2 hv = __floats2half2_rn(nxt[8 * c + 2 * j], nxt[8 * c + 2 * j + 1]);
+          w[j] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        st_async_v4_b32(dst + 16 * (c ^ xsw), w[0], w[1], w[2], w[3], peer_x_full + 8 * sb);
+      }
       return true;
     };
     // block id of this thread's row in tile t, loaded one tile ahead
@@ -341,11 +349,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       if (tr0 && t < 64) trace[t * 32 + 2] = global_timer_ns();
       if (trace && r == 0 && lane == 0 && t < 64) trace[t * 32 + 21 + warp] = global_timer_ns();
       {
-        const float4* xr = (const float4*)(smem + SM::X_OFF + sb * SM::XB + i * (NH * 4));
+        const uint4* xr = (const uint4*)(smem + SM::X_OFF + sb * SM::XB + i * (NH * 2));
 #pragma unroll
         for (int c = 0; c < CPR; ++c) {
-          const float4 x = xr[c ^ xsw];
-          cur[4 * c] += x.x; cur[4 * c + 1] += x.y; cur[4 * c + 2] += x.z; cur[4 * c + 3] += x.w;
+          const uint4 x = xr[c ^ xsw];
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+            cur[8 * c + 2 * j] += f.x;
+            cur[8 * c + 2 * j + 1] += f.y;
+          }
         }
       }
       if (tr0 && t < 64) trace[t * 32 + 12] = global_timer_ns();
