@@ -492,8 +492,24 @@ static BView bview2(const void* p, long long K, long long rows) { return BView{p
 // on tc_gemm_fp8_kernel (tokens converted to f16 into `f16buf` first) with the
 // matrix's block scales, or, given `dq`, on tc_gemm_kernel after dequantising
 // the weight into it.
+static int wgemm_body(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int bn, int splits, void* f16buf,
+                      char* dq, cudaStream_t s);
+
+// Kernel-timer names of the decode weight GEMMs (mla_set_kernel_timer).
+static const char* wgemm_name(WSel w) {
+  return w == W_1 ? "gemm_w1" : w == W_QB ? "gemm_qb" : w == W_UK ? "gemm_uk" : w == W_UV ? "gemm_uv" : "gemm_o";
+}
+
 static int wgemm(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int bn, int splits, void* f16buf,
                  char* dq, cudaStream_t s) {
+  mla_timer_begin(wgemm_name(w), s);
+  const int st = wgemm_body(h, w, bv, g, bn, splits, f16buf, dq, s);
+  mla_timer_end(wgemm_name(w), s);
+  return st;
+}
+
+static int wgemm_body(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int bn, int splits, void* f16buf,
+                      char* dq, cudaStream_t s) {
   const TcState& T = h->tc;
   CUtensorMap B;
   int st;

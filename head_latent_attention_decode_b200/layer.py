@@ -51,11 +51,17 @@ class MlaLayer:
         del src
         self.ws = None
 
-    def __del__(self):
+    def close(self) -> None:
+        """Release the library handle (the weight blob is torch memory)."""
         h = getattr(self, "handle", None)
         if h:
             mla_destroy(h)
             self.handle = None
+
+    def __del__(self):
+        # at interpreter shutdown the module's globals may already be gone
+        if mla_destroy is not None:
+            self.close()
 
     def workspace(self, max_tokens: int, max_context_len: int = 1) -> torch.Tensor:
         need = mla_workspace_bytes(self.handle, max(1, max_tokens), max(1, max_context_len))

@@ -310,10 +310,13 @@ const char* mla_strerror(int status);
 uint64_t mla_kernel_launch_count(void);
 
 /* Kernel timer (tracing). While set, every launch of the library kernel named
- * `kernel` (one of "attn", "front", "gemm", "prefill_attn"; NULL clears the
- * timer) is bracketed by records of the two events (cudaEvent_t, created by
+ * `kernel` is bracketed by records of the two events (cudaEvent_t, created by
  * the caller with timing enabled) on the launch stream, so that
- * cudaEventElapsedTime(start, stop) is that kernel's device time. Inside a
+ * cudaEventElapsedTime(start, stop) is that kernel's device time. Names:
+ * "attn" (decode attention), "prefill_attn", and the decode weight GEMMs
+ * "gemm_w1" (down-projection), "gemm_qb" (wq_b), "gemm_uk" (absorption),
+ * "gemm_uv" (V extraction), "gemm_o" (o_proj), each including the operand
+ * conversion or weight dequantisation it launches. NULL clears the timer. Inside a
  * stream capture the records become external event-record nodes of the graph.
  * Process-wide; not thread-safe against concurrent launches. */
 int mla_set_kernel_timer(const char* kernel, void* start_event, void* stop_event);
