@@ -696,7 +696,8 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     mla_count_launch(1);
   } else if (latent_ok && H <= 128) {
     // (sequence, split) clusters: about three waves of CTA pairs, at most the
-    // splits the workspace holds
+    // splits the workspace holds (six waves balanced random context lengths
+    // better, but the merge's re-read of the extra partials cost as much)
     const int pairs = T.num_sms / 2 > 0 ? T.num_sms / 2 : 74;
     int sp = (int)cdiv(3 * pairs, n);
     if (sp > splits) sp = splits;
@@ -724,7 +725,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
       attr[dev] = true;
     }
     mla_timer_begin("attn", s);
-    launch_pdl(tc_attn_decode_kernel, 2 * n * sp, 320, AttnSmem::SIZE, s, mqp, mc, ml, ta);
+    launch_pdl(tc_attn_decode_kernel, 2 * n * sp, ATT_THREADS, AttnSmem::SIZE, s, mqp, mc, ml, ta);
     mla_timer_end("attn", s);
     mla_count_launch(1);
   } else {
