@@ -40,13 +40,23 @@ def _rope(v, pos, theta, inv_freq=None):
     return out
 
 
+def _softmax_row(s, sink=None):
+    """exp(s_j - m) / (sum_k exp(s_k - m) [+ exp(sink - m)]), m the largest of
+    the row and the sink."""
+    mx = max(s) if sink is None else max(max(s), sink)
+    e = [math.exp(v - mx) for v in s]
+    z = sum(e) + (0.0 if sink is None else math.exp(sink - mx))
+    return [v / z for v in e]
+
+
 def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens,
-                slot_mapping, layout=0, input_norm_w=None, inv_freq=None):
+                slot_mapping, layout=0, input_norm_w=None, inv_freq=None, attn_sink=None):
     """One whole decode step, loops only.
 
     input_norm_w: optional input RMSNorm gamma [hidden] applied to each token
     first (eps = norm_eps); inv_freq: optional RoPE frequency table [d_r/2]
-    replacing theta^(-2i/d_r).
+    replacing theta^(-2i/d_r); attn_sink: optional per-head logit that joins
+    each head's softmax denominator and carries no value.
     cache_rows: list of flat cache rows (lists of R floats), mutated copy returned.
     Returns (out [n][hidden], head_out [n][H][d_v], q_abs [n][H][r_kv],
     q_pe [n][H][d_r], new cache_rows).
@@ -95,10 +105,8 @@ def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens
             s = [(sum(q_abs_all[t][h][cc] * ctx[j][0][cc] for cc in range(rkv))
                   + sum(q_pe_all[t][h][i] * ctx[j][1][i] for i in range(dr))) * scale
                  for j in range(L)]
-            mx = max(s)
-            e = [math.exp(v - mx) for v in s]
-            z = sum(e)
-            o_lat = [sum(e[j] / z * ctx[j][0][cc] for j in range(L)) for cc in range(rkv)]
+            p = _softmax_row(s, None if attn_sink is None else float(attn_sink[h]))
+            o_lat = [sum(p[j] * ctx[j][0][cc] for j in range(L)) for cc in range(rkv)]
             o_t.append([sum(o_lat[cc] * wkv_b[cc][h * (dn + dv) + dn + d] for cc in range(rkv))
                         for d in range(dv)])
         head_out.append(o_t)
@@ -107,9 +115,9 @@ def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens
     return out, head_out, q_abs_all, q_pe_all, rows
 
 
-def prefill(cfg, W, hidden):
-    """Causal expanded prefill of one sequence at positions 0..S-1, loops only.
-    Returns (out [S][hidden], head_out [S][H][d_v])."""
+def prefill(cfg, W, hidden, attn_sink=None):
+    """Causal expanded prefill of one sequence at positions 0..S-1, loops only
+    (attn_sink as in decode_step). Returns (out [S][hidden], head_out [S][H][d_v])."""
     H, dn, dr, dv = cfg.n_heads, cfg.qk_nope, cfg.qk_rope, cfg.v_dim
     rkv = cfg.kv_lora_rank
     S = len(hidden)
@@ -142,11 +150,33 @@ def prefill(cfg, W, hidden):
         o_i = []
         for h in range(H):
             s = [sum(Q[i][h][d] * K[j][h][d] for d in range(dn + dr)) * scale for j in range(i + 1)]
-            mx = max(s)
-            e = [math.exp(v - mx) for v in s]
-            z = sum(e)
-            o_i.append([sum(e[j] / z * V[j][h][d] for j in range(i + 1)) for d in range(dv)])
+            p = _softmax_row(s, None if attn_sink is None else float(attn_sink[h]))
+            o_i.append([sum(p[j] * V[j][h][d] for j in range(i + 1)) for d in range(dv)])
         head_out.append(o_i)
     wo = _mat(W["wo"])
     out = [_vecmat([v for h in range(H) for v in head_out[i][h]], wo) for i in range(S)]
     return out, head_out
+
+
+def v4_qkv(cfg, W, hidden, positions, kv_norm_w, inv_freq=None):
+    """DeepSeek-V4 QKV projection, loops only (same reading as mla_ref.v4_qkv:
+    per-head root-mean-square norm without gain, interleaved RoPE on the last
+    d_r of each head and of the kv row, kv RMSNorm over all its columns).
+    Returns (q [n][H][hd], kv [n][kv_dim])."""
+    H, hd, dr = cfg.n_heads, cfg.qk_nope + cfg.qk_rope, cfg.qk_rope
+    qs, kvs = [], []
+    for t, x in enumerate(hidden):
+        x = [float(v) for v in x]
+        pos = int(positions[t])
+        ql = _rms(_vecmat(x, _mat(W["wq_a"])), [float(g) for g in W["q_norm_w"]], cfg.norm_eps)
+        q = _vecmat(ql, _mat(W["wq_b"]))
+        q_t = []
+        for h in range(H):
+            qh = q[h * hd:(h + 1) * hd]
+            qh = _rms(qh, [1.0] * hd, cfg.norm_eps)
+            q_t.append(qh[:hd - dr] + _rope(qh[hd - dr:], pos, cfg.rope_theta, inv_freq))
+        kv = _rms(_vecmat(x, _mat(W["wkv_a"])), [float(g) for g in kv_norm_w], cfg.norm_eps)
+        R = len(kv)
+        kvs.append(kv[:R - dr] + _rope(kv[R - dr:], pos, cfg.rope_theta, inv_freq))
+        qs.append(q_t)
+    return qs, kvs

@@ -89,6 +89,23 @@ def softmax(s, axis=-1):
     return e / np.sum(e, axis=axis, keepdims=True)
 
 
+def softmax_with_sink(s, sink):
+    """Softmax over the last axis with one extra logit per row that carries no
+    value: p_j = e^{s_j} / (sum_k e^{s_k} + e^{sink}).
+
+    "Struct MlaWeights", attn_sink: a per-head attention sink logit (DeepSeek-V4
+    s_aux). The page gives only that it is one logit per query head. Reading
+    adopted: the sink is one more column of the softmax, in the units of the
+    scaled scores, and its own probability is dropped, so a head's weights sum
+    to less than one. Written as exactly that: the plain softmax of the row
+    extended by the sink, without its last column.
+    """
+    s = np.asarray(s, np.float64)
+    sink = np.broadcast_to(np.asarray(sink, np.float64), s.shape[:-1])
+    full = np.concatenate([s, sink[..., None]], axis=-1)
+    return softmax(full, axis=-1)[..., :-1]
+
+
 def softmax_scale(qk_nope, qk_rope, mscale=1.0):
     """1/sqrt(qk_nope + qk_rope) * mscale^2.
 
@@ -298,7 +315,7 @@ def decode_qkv(cfg, W, hidden, cos, sin, kv_cache, slot_mapping, row_layout=LATE
 
 
 def decode_attn(cfg, W, q_abs, q_pe, kv_cache, block_table, context_lens,
-                row_layout=LATENT_FIRST, scale=None):
+                row_layout=LATENT_FIRST, scale=None, attn_sink=None):
     """Absorbed attention over the latent cache, V extraction and o_proj.
 
     For token t (sequence t) with L = context_lens[t] rows:
@@ -306,7 +323,9 @@ def decode_attn(cfg, W, q_abs, q_pe, kv_cache, block_table, context_lens,
       p = softmax_j(s);  o_lat[h] = sum_j p[h, j] c_j;  o[h] = o_lat[h] @ W_UV[h]
       out = concat_h(o[h]) @ wo
     "Struct MlaWeights": w_uk_t (absorption), w_uv (v_out = attn_latent @ W_UV),
-    wo; "struct Mla": scale. Returns (out [n, hidden], head_out [n, H, d_v]).
+    wo; "struct Mla": scale. attn_sink [H] (optional): each head's softmax
+    takes the sink logit as one more column (softmax_with_sink).
+    Returns (out [n, hidden], head_out [n, H, d_v]).
     """
     scale = softmax_scale(cfg.qk_nope, cfg.qk_rope) if scale is None else scale
     _, w_uv = split_wkv_b(W["wkv_b"], cfg.n_heads, cfg.qk_nope, cfg.v_dim)
@@ -317,7 +336,7 @@ def decode_attn(cfg, W, q_abs, q_pe, kv_cache, block_table, context_lens,
         c, k_pe = split_row(rows, cfg.kv_lora_rank, row_layout)
         s = (np.asarray(q_abs[t], np.float64) @ c.T
              + np.asarray(q_pe[t], np.float64) @ k_pe.T) * scale           # [H, L]
-        p = softmax(s, axis=-1)
+        p = softmax(s, axis=-1) if attn_sink is None else softmax_with_sink(s, attn_sink)
         o_lat = p @ c                                                      # [H, r_kv]
         head_out[t] = np.einsum("hc,hcd->hd", o_lat, w_uv)
     out = head_out.reshape(n, -1) @ W["wo"]
@@ -352,7 +371,7 @@ def decode_attn_expanded(cfg, W, q_nope, q_pe, kv_cache, block_table, context_le
 # prefill (context encoding): the expanded path
 # ----------------------------------------------------------------------------
 
-def prefill(cfg, W, hidden, cos, sin, rows=None, scale=None, row_layout=LATENT_FIRST):
+def prefill(cfg, W, hidden, cos, sin, rows=None, scale=None, row_layout=LATENT_FIRST, attn_sink=None):
     """Causal prefill of one sequence with K/V expanded from the latent.
 
     "QKV CTE MLA Kernel API Reference", qkv_mla_mx Notes: Stage 1 x @ [wq_a | wkv_a]
@@ -360,6 +379,8 @@ def prefill(cfg, W, hidden, cos, sin, rows=None, scale=None, row_layout=LATENT_F
     norm(kv) @ wkv_b split per head into k_nope, v; Final assembly: RoPE on q_pe
     and k_pe, k_pe broadcast to all heads and concatenated with k_nope. Then
     causal softmax(Q K^T * scale) V (query i sees keys j <= i) and o_proj.
+    attn_sink [H] (optional): each head's softmax takes the sink logit as one
+    more column (softmax_with_sink).
 
     rows: query rows to evaluate (default all). K/V are always built for all S
     tokens. Returns (out [len(rows), hidden], head_out [len(rows), H, d_v],
@@ -379,10 +400,53 @@ def prefill(cfg, W, hidden, cos, sin, rows=None, scale=None, row_layout=LATENT_F
         i = int(i)
         s = (np.einsum("hp,jhp->hj", q_nope[m], k_nope[:i + 1])
              + q_pe[m] @ k_pe[:i + 1].T) * scale                       # [H, i+1]
-        p = softmax(s, axis=-1)
+        p = softmax(s, axis=-1) if attn_sink is None else softmax_with_sink(s, attn_sink)
         head_out[m] = np.einsum("hj,jhd->hd", p, v[:i + 1])
     out = head_out.reshape(len(rows), -1) @ np.asarray(W["wo"], np.float64)
     return out, head_out, cache_row(c, k_pe, row_layout)
+
+
+# ----------------------------------------------------------------------------
+# DeepSeek-V4 QKV projection
+# ----------------------------------------------------------------------------
+
+def head_rms(q, eps):
+    """Each head's vector divided by the root of its mean square (+ eps), no gain:
+    the "per-head rsqrt norm" of "QKV CTE MLA Kernel API Reference",
+    qkv_mla_mx_deepseek_v4, Final assembly. Reading adopted: the RMS form of
+    the norm used everywhere else on the pages, with the kernel's norm_eps."""
+    q = np.asarray(q, np.float64)
+    return q / np.sqrt(np.mean(q * q, axis=-1, keepdims=True) + eps)
+
+
+def v4_qkv(cfg, W, hidden, cos, sin, kv_norm_w):
+    """(q [n, H, hd], kv [n, kv_dim]) of the DeepSeek-V4 QKV projection.
+
+    "QKV CTE MLA Kernel API Reference", qkv_mla_mx_deepseek_v4, Notes:
+      fused first projection x @ wqkv [H_in, qk_lora_rank + kv_dim], split into
+      qr [qk_lora_rank] and kv [kv_dim] (kv_dim = kv_lora_rank + qk_rope);
+      Q stage 2: norm(qr) @ wq_b [qk_lora_rank, n_heads * head_dim], with the
+      q_norm gamma;
+      final assembly: q -> per-head rsqrt norm -> RoPE on the last qk_rope dims
+      of each head; kv -> RMSNorm with kv_norm_gamma [kv_dim] over all kv_dim
+      columns -> RoPE on its last qk_rope columns (the kv latent is returned).
+    Here wqkv is [wq_a | wkv_a] (the same fused first projection this library
+    already uses), head_dim = qk_nope + qk_rope, and kv_norm_w has kv_dim
+    entries. Readings: RoPE is the interleaved pairing of the decode page; the
+    per-head norm is head_rms.
+    """
+    x = np.asarray(hidden, np.float64)
+    eps = cfg.norm_eps
+    H, hd, dr = cfg.n_heads, cfg.qk_nope + cfg.qk_rope, cfg.qk_rope
+    qr = x @ np.asarray(W["wq_a"], np.float64)
+    kv = x @ np.asarray(W["wkv_a"], np.float64)
+    q = (rms_norm(qr, W["q_norm_w"], eps) @ np.asarray(W["wq_b"], np.float64)).reshape(x.shape[0], H, hd)
+    q = head_rms(q, eps)
+    q[..., hd - dr:] = rope_interleaved(q[..., hd - dr:], cos[:, None, :], sin[:, None, :])
+    kv = rms_norm(kv, kv_norm_w, eps)
+    R = kv.shape[1]
+    kv[:, R - dr:] = rope_interleaved(kv[:, R - dr:], cos, sin)
+    return q, kv
 
 
 # ----------------------------------------------------------------------------
