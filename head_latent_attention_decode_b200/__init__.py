@@ -37,6 +37,7 @@ SYMBOLS = (
     "mla_decode_qkv", "mla_decode_attn", "mla_prefill", "mla_strerror",
     "mla_kernel_launch_count", "mla_set_kernel_timer", "mla_decode_qkv_noalloc",
     "mla_decode_step_host_bytes", "mla_decode_step_host", "mla_rope_cos_sin_inv_freq",
+    "mla_v4_qkv",
 )
 
 MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -52,7 +53,7 @@ class mla_config(ctypes.Structure):
 class mla_weights_desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "wq_a", "wq_b", "wkv_a", "wkv_b", "wo", "q_norm_w", "kv_norm_w", "wq_a_scale",
-        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale")]
+        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale", "attn_sink")]
 
 
 class MlaError(RuntimeError):
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_attn.argtypes = [vp, vp, vp, vp, i, vp, i, vp, i, i, vp, vp, vp, sz, vp]
         L.mla_prefill.restype = i
         L.mla_prefill.argtypes = [vp, vp, i, vp, vp, vp, vp, vp, i, vp, vp, sz, vp]
+        L.mla_v4_qkv.restype = i
+        L.mla_v4_qkv.argtypes = [vp, vp, i, vp, vp, vp, vp, vp, vp, sz, vp]
         L.mla_strerror.restype = ctypes.c_char_p
         L.mla_strerror.argtypes = [i]
         L.mla_kernel_launch_count.restype = ctypes.c_uint64
@@ -157,10 +160,10 @@ def mla_weights_bytes(cfg: mla_config) -> int:
 
 def mla_init_weights(cfg: mla_config, weights: dict, dst: torch.Tensor, stream=None) -> int:
     """weights: name -> device tensor (wq_a, wq_b, wkv_a, wkv_b, wo, q_norm_w, kv_norm_w,
-    and *_scale for FP8). Returns the opaque handle (int)."""
+    *_scale for FP8, optional attn_sink [H] fp32). Returns the opaque handle (int)."""
     d = mla_weights_desc(*[_ptr(weights.get(n)) for n in (
         "wq_a", "wq_b", "wkv_a", "wkv_b", "wo", "q_norm_w", "kv_norm_w", "wq_a_scale",
-        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale")])
+        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale", "attn_sink")])
     h = ctypes.c_void_p()
     _check(lib().mla_init_weights(ctypes.byref(cfg), ctypes.byref(d), _ptr(dst), _nbytes(dst),
                                   _stream(stream), ctypes.byref(h)), "mla_init_weights")
@@ -261,6 +264,14 @@ def mla_prefill(handle, hidden, cos, sin, out, ws, head_out=None, kv_cache=None,
                              kv_cache.shape[0] if kv_cache is not None else 0,
                              _ptr(slot_mapping), _ptr(ws), _nbytes(ws), _stream(stream)),
            "mla_prefill")
+
+
+def mla_v4_qkv(handle, hidden, cos, sin, kv_norm_w, q_out, kv_out, ws, stream=None) -> None:
+    """DeepSeek-V4 QKV projection (see include/mla.h): q_out [S, H, d_n + d_r],
+    kv_out [S, r_kv + d_r]."""
+    S = hidden.shape[0]
+    _check(lib().mla_v4_qkv(handle, _ptr(hidden), S, _ptr(cos), _ptr(sin), _ptr(kv_norm_w), _ptr(q_out),
+                            _ptr(kv_out), _ptr(ws), _nbytes(ws), _stream(stream)), "mla_v4_qkv")
 
 
 def mla_kernel_launch_count() -> int:

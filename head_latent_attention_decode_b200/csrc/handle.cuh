@@ -34,7 +34,7 @@ void mla_timer_end(const char* kernel, cudaStream_t s);
 struct WeightLayout {
   int Nq1, N1, R, Hq, Hkv;
   size_t esz;
-  size_t W1, Wqb, Wuk, Wuv, Wkvb, Wo, gq, gkv;
+  size_t W1, Wqb, Wuk, Wuv, Wkvb, Wo, gq, gkv, sink;
   size_t sW1, sWqb, sWuk, sWuv, sWkvb, sWo;
   size_t total;
 };
@@ -44,6 +44,7 @@ struct mla_handle {
   WeightLayout L;
   float scale;
   char* base;
+  int has_sink;   // attn_sink given at init: one fp32 logit per head at base + L.sink
   int device;
   TcState tc;
   // mla_decode_step_host: page-locked packing buffer for the step's int32

@@ -88,6 +88,7 @@ static WeightLayout make_layout(const mla_config* c) {
   L.Wo = put((size_t)D * H * dv * L.esz);
   L.gq = rq ? put((size_t)rq * 4) : 0;
   L.gkv = put((size_t)rkv * 4);
+  L.sink = put((size_t)H * 4);
   if (fp8) {
     L.sW1 = put(sblocks(L.N1, D));
     L.sWqb = rq ? put(sblocks(L.Hq, rq)) : 0;
@@ -301,6 +302,8 @@ int mla_init_weights(const mla_config* cfg, const mla_weights_desc* w, void* dst
   gather(L.Wo, w->wo, 0, 0, 1, D, 1, D, H * dv, e);
   if (rq) cudaMemcpyAsync(h->base + L.gq, w->q_norm_w, (size_t)rq * 4, cudaMemcpyDeviceToDevice, s);
   cudaMemcpyAsync(h->base + L.gkv, w->kv_norm_w, (size_t)rkv * 4, cudaMemcpyDeviceToDevice, s);
+  h->has_sink = w->attn_sink != nullptr;
+  if (w->attn_sink) cudaMemcpyAsync(h->base + L.sink, w->attn_sink, (size_t)H * 4, cudaMemcpyDeviceToDevice, s);
   if (fp8) {
     // scale tensors [ceil(in/128), ceil(out/128)] -> per K-major matrix [N/128][K/128]
     const long long Db = cdiv(D, 128), Rb = cdiv(L.R, 128), Hqb = L.Hq / 128, rqb = rq / 128;
@@ -491,8 +494,9 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
     mla_timer_end("attn", s);
     count_launch();
     dim3 cg(n, H);
-    if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat);
-    else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat);
+    const float* sink = h->has_sink ? (const float*)(h->base + L.sink) : nullptr;
+    if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat, sink);
+    else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat, sink);
     count_launch();
   }
   // head_out[h] = o_lat[h] @ W_UV[h]
@@ -709,6 +713,7 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos, cons
   pa.Q = Q; pa.ldq = L.Hq; pa.KV = KV; pa.ldkv = L.Hkv; pa.kpe = wsb + W.pkpe;
   pa.O = head; pa.ldo = (long long)H * dv; pa.S = S; pa.H = H; pa.d_n = dn; pa.d_r = dr; pa.d_v = dv;
   pa.scale = h->scale;
+  pa.sink = h->has_sink ? (const float*)(h->base + L.sink) : nullptr;
   const size_t smem = (size_t)(PA_BQ * (dn + dr) + PA_BK * (dn + dr + 1) + PA_BK * dv) * 4;
   dim3 grid((unsigned)cdiv(S, PA_BQ), H);
   mla_timer_begin("prefill_attn", s);
@@ -718,6 +723,47 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos, cons
   count_launch();
   launch_linear(ta, tw, ta, lin(head, (long long)H * dv, h->base + L.Wo, (long long)H * dv, wscale(h, L.sWo),
                                 cdiv((long long)H * dv, 128), out, D, S, D, H * dv), 1, s);
+  return cuda_status();
+}
+
+int mla_v4_qkv(mla_handle* h, const void* hidden, int S, const float* cos, const float* sin,
+               const float* kv_norm_w, void* q_out, void* kv_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!h || S < 0) return MLA_ERR_INVALID_ARG;
+  if (S == 0) return MLA_OK;
+  if (!hidden || !cos || !sin || !kv_norm_w || !q_out || !kv_out || !ws) return MLA_ERR_INVALID_ARG;
+  const mla_config* c = &h->cfg;
+  if (c->q_lora_rank == 0) return MLA_ERR_UNSUPPORTED;   // the V4 query path is low-rank
+  const WsLayout W = make_ws(h, S, 1);
+  if (ws_bytes < W.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* wsb = (char*)ws;
+  int* flag = (int*)wsb;
+  const WeightLayout& L = h->L;
+  const int H = c->n_heads, dn = c->qk_nope, dr = c->qk_rope, rkv = c->kv_lora_rank;
+  const int D = c->hidden, rq = c->q_lora_rank;
+  const int ta = acode(h), tw = wcode(h);
+  if (tc_prefill_supported(h, S)) {
+    const int r = tc_v4_qkv(h, hidden, S, cos, sin, kv_norm_w, q_out, kv_out, wsb, W.pY1, W.pqn, W.pDQ, s);
+    return r != MLA_OK ? r : cuda_status();
+  }
+  float* Y1 = (float*)(wsb + W.pY1);
+  launch_linear(ta, tw, 0, lin(hidden, D, h->base + L.W1, D, wscale(h, L.sW1), cdiv(D, 128), Y1, L.N1, S, L.N1, D), 1, s);
+  FrontFoldArgs f{};
+  f.Y = Y1; f.ldy = L.N1; f.kv0 = L.Nq1;
+  f.r_q = rq; f.r_kv = rkv; f.d_r = dr;
+  f.q_norm_w = (const float*)(h->base + L.gq);
+  f.kv_norm_w = kv_norm_w; f.eps = c->norm_eps;
+  f.cos = cos; f.sin = sin;
+  f.qn = wsb + W.pqn; f.ldqn = rq;
+  f.cache = kv_out; f.n_rows = S; f.slot = nullptr; f.layout = MLA_ROW_LATENT_FIRST; f.flag = flag;
+  f.v4 = 1;
+  if (ta == 0) frontfold_epilogue_kernel<float><<<S, 256, 0, s>>>(f);
+  else frontfold_epilogue_kernel<bf16><<<S, 256, 0, s>>>(f);
+  count_launch();
+  launch_linear(ta, tw, ta, lin(wsb + W.pqn, rq, h->base + L.Wqb, rq, wscale(h, L.sWqb), rq / 128, q_out, L.Hq, S, L.Hq, rq), 1, s);
+  if (ta == 0) q_headnorm_rope_kernel<float><<<S, 256, 0, s>>>((float*)q_out, L.Hq, H, dn + dr, dr, cos, sin, c->norm_eps);
+  else q_headnorm_rope_kernel<bf16><<<S, 256, 0, s>>>((bf16*)q_out, L.Hq, H, dn + dr, dr, cos, sin, c->norm_eps);
+  count_launch();
   return cuda_status();
 }
 

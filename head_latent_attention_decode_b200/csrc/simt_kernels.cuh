@@ -120,6 +120,10 @@ struct FrontFoldArgs {
   const int* slot; int layout;
   void* cn; void* kpe;                    // prefill: [n, r_kv], [n, d_r] act
   int* flag;
+  // DeepSeek-V4 form ("QKV CTE MLA Kernel API Reference", qkv_mla_mx_deepseek_v4):
+  // the whole kv row [r_kv + d_r] is RMS-normed with a gamma of that length and
+  // its normed tail is rotated; with slot == NULL row t goes to cache row t
+  int v4;
 };
 
 template <typename TACT>
@@ -137,13 +141,14 @@ __global__ void __launch_bounds__(256) frontfold_epilogue_kernel(FrontFoldArgs p
     for (int i = threadIdx.x; i < p.r_q; i += blockDim.x) q[i] = from_f32<TACT>(y[i] * r * p.q_norm_w[i]);
   }
   const float* kv = y + p.kv0;
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < p.r_kv; i += blockDim.x) ss += kv[i] * kv[i];
-  const float r = rsqrtf(block_sum(ss, red) / (float)p.r_kv + p.eps);
   const int R = p.r_kv + p.d_r;
+  const int nn = p.v4 ? R : p.r_kv;       // the normed width
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) ss += kv[i] * kv[i];
+  const float r = rsqrtf(block_sum(ss, red) / (float)nn + p.eps);
   TACT* row = nullptr;
   if (p.cache) {
-    const int s = p.slot[t];
+    const int s = p.slot ? p.slot[t] : t;
     if (s >= 0 && (long long)s < p.n_rows) {
       row = (TACT*)p.cache + (long long)s * R;
     } else if (s >= 0) {
@@ -160,8 +165,13 @@ __global__ void __launch_bounds__(256) frontfold_epilogue_kernel(FrontFoldArgs p
   const float* pe = kv + p.r_kv;
   const int half = p.d_r / 2;
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    float e0 = pe[2 * i], e1 = pe[2 * i + 1];
+    if (p.v4) {
+      e0 *= r * p.kv_norm_w[p.r_kv + 2 * i];
+      e1 *= r * p.kv_norm_w[p.r_kv + 2 * i + 1];
+    }
     float o0, o1;
-    rope_pair(pe[2 * i], pe[2 * i + 1], p.cos[(long long)t * half + i], p.sin[(long long)t * half + i], &o0, &o1);
+    rope_pair(e0, e1, p.cos[(long long)t * half + i], p.sin[(long long)t * half + i], &o0, &o1);
     const TACT a = from_f32<TACT>(o0), b = from_f32<TACT>(o1);
     if (row) { row[pe_off + 2 * i] = a; row[pe_off + 2 * i + 1] = b; }
     if (p.kpe) {
@@ -188,6 +198,40 @@ __global__ void q_rope_kernel(const TQ* Q, long long ldq, int H, int d_n, int d_
     TOUT* o = out + (long long)t * ldo + (long long)h * out_head_stride + out_off;
     o[2 * i] = from_f32<TOUT>(o0);
     o[2 * i + 1] = from_f32<TOUT>(o1);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// DeepSeek-V4 query heads, in place: each head of q [n, H, hd] (row stride ldq)
+// is divided by the root of its mean square (+ eps, no gain), then its last
+// d_r entries are rotated by interleaved RoPE at the token's position
+// ("QKV CTE MLA Kernel API Reference", qkv_mla_mx_deepseek_v4, Final assembly:
+// per-head rsqrt norm, then RoPE on the last rope dims). grid n, 256 threads:
+// warp w handles heads w, w + 8, ...
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) q_headnorm_rope_kernel(T* q, long long ldq, int H, int hd, int d_r,
+                                                              const float* cos, const float* sin, float eps) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = d_r / 2, base = hd - d_r;
+  for (int h = warp; h < H; h += (int)(blockDim.x >> 5)) {
+    T* qh = q + (long long)t * ldq + (long long)h * hd;
+    float ss = 0.f;
+    for (int j = lane; j < hd; j += 32) {
+      const float v = to_f32(qh[j]);
+      ss += v * v;
+    }
+    const float r = rsqrtf(warp_sum(ss) / (float)hd + eps);   // every lane has read its entries
+    for (int j = lane; j < base; j += 32) qh[j] = from_f32<T>(to_f32(qh[j]) * r);
+    for (int i = lane; i < half; i += 32) {
+      float o0, o1;
+      rope_pair(to_f32(qh[base + 2 * i]) * r, to_f32(qh[base + 2 * i + 1]) * r, cos[(long long)t * half + i],
+                sin[(long long)t * half + i], &o0, &o1);
+      qh[base + 2 * i] = from_f32<T>(o0);
+      qh[base + 2 * i + 1] = from_f32<T>(o1);
+    }
   }
 }
 
@@ -300,11 +344,13 @@ __global__ void __launch_bounds__(256) attn_decode_simt_kernel(AttnArgs p) {
 }
 
 // Merge split partials: o_lat = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s.
-// grid (n, H), 128 threads x 4 consecutive columns (r_kv <= 512, r_kv % 4 == 0).
-// Writes o_lat [n, H, r_kv] in act dtype.
+// With a per-head sink logit z_h ("Struct MlaWeights", attn_sink) the softmax
+// has one more column that carries no value: M also covers z_h and the
+// denominator gains e^{z_h - M}. grid (n, H), 128 threads x 4 consecutive
+// columns (r_kv <= 512, r_kv % 4 == 0). Writes o_lat [n, H, r_kv] in act dtype.
 template <typename T>
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, const float* part_ml, int n_splits,
-                                                           int H, int r_kv, T* o_lat) {
+                                                           int H, int r_kv, T* o_lat, const float* sink) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ float wsh[64];
@@ -317,7 +363,9 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, 
       if (part_ml[base * 2 + 1] > 0.f) M = fmaxf(M, part_ml[base * 2]);
     }
     M = warp_max(M);
-    float den = 0.f;
+    const float z = sink ? sink[h] : -INFINITY;
+    M = fmaxf(M, z);
+    float den = (threadIdx.x == 0 && z > -INFINITY) ? __expf(z - M) : 0.f;
     for (int s = threadIdx.x; s < n_splits; s += 32) {
       const long long base = ((long long)t * n_splits + s) * H + h;
       const float l = part_ml[base * 2 + 1];
@@ -364,6 +412,7 @@ struct PrefillAttnArgs {
   void* O; long long ldo;                // [S, H*d_v]
   int S, H, d_n, d_r, d_v;
   float scale;
+  const float* sink;                     // [H] sink logits (one more softmax column, no value), or NULL
 };
 
 constexpr int PA_BQ = 32, PA_BK = 32;
@@ -445,7 +494,8 @@ __global__ void __launch_bounds__(128) prefill_attn_simt_kernel(PrefillAttnArgs 
   for (int q = 0; q < 8; ++q) {
     const int i = i0 + warp * 8 + q;
     if (i >= p.S) continue;
-    const float inv = l[q] > 0.f ? 1.f / l[q] : 0.f;
+    const float den = l[q] + ((p.sink && l[q] > 0.f) ? __expf(p.sink[h] - m[q]) : 0.f);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
       if (c < per_lane) O[(long long)i * p.ldo + (long long)h * p.d_v + lane + 32 * c] = from_f32<T>(o[q][c] * inv);

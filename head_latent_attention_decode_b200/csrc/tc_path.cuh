@@ -742,7 +742,9 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     mla_timer_end("attn", s);
     mla_count_launch(1);
   }
-  launch_pdl(attn_combine_kernel<bf16>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits, H, rkv, o_lat);
+  const float* sink = h->has_sink ? (const float*)(h->base + h->L.sink) : nullptr;
+  launch_pdl(attn_combine_kernel<bf16>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits, H,
+             rkv, o_lat, sink);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -773,6 +775,56 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   const long long cnt = (long long)n * D;
   launch_pdl(splitk_reduce_bf16_kernel, (unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s,
              (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);
+  mla_count_launch(1);
+  return MLA_OK;
+}
+
+// DeepSeek-V4 QKV projection on the prefill tensor-core GEMMs ("QKV CTE MLA
+// Kernel API Reference", qkv_mla_mx_deepseek_v4): Y1 = x @ [wq_a | wkv_a]
+// (fp32), the front-fold in its V4 form (q latent RMSNorm -> qn; the whole kv
+// row RMS-normed with kv_norm_w [r_kv + d_r], its tail rotated -> kv_out),
+// q = qn @ wq_b written as bf16 into q_out, then each head normalised without
+// gain and its tail rotated in place. FP8 handles dequantise each weight first.
+static inline int tc_v4_qkv(const mla_handle* h, const void* hidden, int S, const float* cos, const float* sin,
+                            const float* kv_norm_w, void* q_out, void* kv_out, char* ws, size_t pY1, size_t pqn,
+                            size_t pDQ, cudaStream_t s) {
+  const mla_config& c = h->cfg;
+  const WeightLayout& L = h->L;
+  const TcState& T = h->tc;
+  int* flag = (int*)ws;
+  const int H = c.n_heads, dn = c.qk_nope, dr = c.qk_rope, rkv = c.kv_lora_rank, D = c.hidden;
+  const int rq = c.q_lora_rank;
+  int st;
+  char* dq = T.pf8 ? ws + pDQ : nullptr;
+  const int sop = T.pf8 ? 0 : 2;
+  CUtensorMap mx;
+  if ((st = make_map2(&mx, hidden, D, S, D, 128)) != MLA_OK) return st;
+  float* Y1 = (float*)(ws + pY1);
+  GemmArgs g = gemm_args(S, L.N1, D, 1, EPI_F32_N, Y1, L.N1, 0, flag);
+  CUtensorMap bw;
+  if ((st = prefill_weight_map(h, &bw, T.b_W1, L.W1, L.sW1, L.N1, D, 0, L.N1, dq, true, s)) != MLA_OK) return st;
+  g.static_op = sop;
+  if ((st = launch_gemm(mx, bw, g, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+  FrontFoldArgs f{};
+  f.Y = Y1; f.ldy = L.N1; f.kv0 = L.Nq1;
+  f.r_q = rq; f.r_kv = rkv; f.d_r = dr;
+  f.q_norm_w = (const float*)(h->base + L.gq);
+  f.kv_norm_w = kv_norm_w; f.eps = c.norm_eps;
+  f.cos = cos; f.sin = sin;
+  f.qn = ws + pqn; f.ldqn = rq;
+  f.cache = kv_out; f.n_rows = S; f.slot = nullptr; f.layout = MLA_ROW_LATENT_FIRST; f.flag = flag;
+  f.v4 = 1;
+  launch_pdl(frontfold_epilogue_kernel<bf16>, S, 256, 0, s, f);
+  mla_count_launch(1);
+  CUtensorMap mq;
+  if ((st = make_map2(&mq, ws + pqn, rq, S, rq, 128)) != MLA_OK) return st;
+  GemmArgs g2 = gemm_args(S, L.Hq, rq, 1, EPI_BF16_N, q_out, L.Hq, 0, flag);
+  CUtensorMap bq;
+  if ((st = prefill_weight_map(h, &bq, T.b_Wqb, L.Wqb, L.sWqb, L.Hq, rq, 0, L.Hq, dq, true, s)) != MLA_OK) return st;
+  g2.static_op = sop;
+  if ((st = launch_gemm(mq, bq, g2, 256, 1, T.num_sms, s)) != MLA_OK) return st;
+  launch_pdl(q_headnorm_rope_kernel<bf16>, S, 256, 0, s, (bf16*)q_out, (long long)L.Hq, H, dn + dr, dr, cos, sin,
+             c.norm_eps);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -856,6 +908,7 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
     pa.S = S; pa.H = H; pa.q_tiles = (int)cdiv(S, 128);
     pa.scale_log2 = h->scale * 1.4426950408889634f;
     pa.out = (bf16*)head; pa.flag = flag;
+    pa.sink = h->has_sink ? (const float*)(h->base + L.sink) : nullptr;
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -872,6 +925,7 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
     pa.Q = Q; pa.ldq = L.Hq; pa.KV = KV; pa.ldkv = L.Hkv; pa.kpe = ws + pkpe;
     pa.O = head; pa.ldo = (long long)H * dv; pa.S = S; pa.H = H; pa.d_n = dn; pa.d_r = dr; pa.d_v = dv;
     pa.scale = h->scale;
+    pa.sink = h->has_sink ? (const float*)(h->base + L.sink) : nullptr;
     const size_t smem = (size_t)(PA_BQ * (dn + dr) + PA_BK * (dn + dr + 1) + PA_BK * dv) * 4;
     cudaFuncSetAttribute(prefill_attn_simt_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     mla_timer_begin("prefill_attn", s);

@@ -29,6 +29,7 @@ struct TcPrefillAttnArgs {
   float scale_log2;
   bf16* out;          // [S, H * 128]
   int* flag;
+  const float* sink;  // [H] sink logits (one more softmax column, no value), or NULL
 };
 
 struct PaSmem {
@@ -329,7 +330,9 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(lx_b);
       if (mbar_wait_warp(lx_b, 0, abort_word, a.flag)) {
-        const float lsum = lx[row] + lx[128 + row];
+        float lsum = lx[row] + lx[128 + row];
+        // a sink logit z joins the denominator as e^z (m_ref is in log2 units of the scaled scores)
+        if (a.sink && lsum > 0.f) lsum += ex2_approx(fmaf(a.sink[h], 1.4426950408889634f, -m_ref));
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         bf16* o_row = a.out + (long long)qi * a.H * 128 + h * 128 + 64 * half;
         for (int c = 0; c < 4; ++c) {

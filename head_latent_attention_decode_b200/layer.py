@@ -9,8 +9,8 @@ import numpy as np
 import torch
 
 from . import (MLA_ROW_LATENT_FIRST, make_config, mla_decode_attn, mla_decode_qkv, mla_destroy,
-               mla_init_weights, mla_prefill, mla_rope_cos_sin, mla_rope_cos_sin_inv_freq, mla_weights_bytes,
-               mla_workspace_bytes, mla_workspace_init)
+               mla_init_weights, mla_prefill, mla_rope_cos_sin, mla_rope_cos_sin_inv_freq, mla_v4_qkv,
+               mla_weights_bytes, mla_workspace_bytes, mla_workspace_init)
 
 ACT_TORCH = {"f32": torch.float32, "bf16": torch.bfloat16}
 
@@ -35,7 +35,7 @@ class MlaLayer:
     """One layer's repacked weights (device) and C-ABI handle."""
 
     def __init__(self, shape, weights, row_layout: int = MLA_ROW_LATENT_FIRST,
-                 device: str = "cuda", softmax_scale: float = 0.0):
+                 device: str = "cuda", softmax_scale: float = 0.0, attn_sink=None):
         self.shape = shape
         self.device = torch.device(device)
         self.act = ACT_TORCH[shape.act_dtype]
@@ -45,7 +45,9 @@ class MlaLayer:
         if nbytes == 0:
             raise ValueError(f"configuration not accepted by the library: {shape}")
         self.blob = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-        src = upload_weights(weights, self.device) if not isinstance(weights, dict) else weights
+        src = upload_weights(weights, self.device) if not isinstance(weights, dict) else dict(weights)
+        if attn_sink is not None:   # per-head sink logits, fp32 [n_heads]
+            src["attn_sink"] = torch.as_tensor(attn_sink, dtype=torch.float32).to(self.device).contiguous()
         self.handle = mla_init_weights(self.cfg, src, self.blob)
         torch.cuda.current_stream(self.device).synchronize()
         del src
@@ -107,6 +109,19 @@ class MlaLayer:
         mla_decode_attn(self.handle, q_abs, q_pe, kv_cache, block_table, context_lens,
                         max_context_len, out, ws, head_out=head_out)
         return out
+
+    def v4_qkv(self, hidden, cos, sin, kv_norm_w, q_out=None, kv_out=None):
+        """DeepSeek-V4 QKV projection: (q [S, H, d_n + d_r], kv [S, r_kv + d_r])."""
+        s = self.shape
+        S = hidden.shape[0]
+        if q_out is None:
+            q_out = torch.empty((S, s.n_heads, s.qk_nope + s.qk_rope), dtype=self.act, device=self.device)
+        if kv_out is None:
+            kv_out = torch.empty((S, s.kv_lora_rank + s.qk_rope), dtype=self.act, device=self.device)
+        ws = self.ws if self.ws is not None and self.ws.numel() >= mla_workspace_bytes(
+            self.handle, max(S, 1), 1) else self.workspace(S, 1)
+        mla_v4_qkv(self.handle, hidden, cos, sin, kv_norm_w, q_out, kv_out, ws)
+        return q_out, kv_out
 
     def prefill(self, hidden, cos, sin, out=None, head_out=None, kv_cache=None, slot_mapping=None):
         s = self.shape

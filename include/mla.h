@@ -101,7 +101,13 @@ typedef struct {
  *   wkv_b [r_kv, H*(d_n+d_v)]       per head [k_nope_h | v_h] columns
  *   wo    [H*d_v, D]
  *   q_norm_w [r_q] fp32 (NULL when q_lora_rank == 0), kv_norm_w [r_kv] fp32
- *   *_scale: FP8 only, fp32 [ceil(in/128), ceil(out/128)], else NULL. */
+ *   *_scale: FP8 only, fp32 [ceil(in/128), ceil(out/128)], else NULL.
+ *   attn_sink [H] fp32 or NULL: a per-head attention sink logit ("Struct
+ *            MlaWeights", attn_sink, DeepSeek-V4 s_aux; a bf16 checkpoint
+ *            value converts to fp32 exactly). When set, every softmax of
+ *            mla_decode_attn and mla_prefill takes it as one more column in
+ *            the units of the scaled scores that carries no value:
+ *            p_j = e^{s_j} / (sum_k e^{s_k} + e^{attn_sink[h]}). */
 typedef struct {
   const void* wq_a;
   const void* wq_b;
@@ -115,6 +121,7 @@ typedef struct {
   const float* wkv_a_scale;
   const float* wkv_b_scale;
   const float* wo_scale;
+  const float* attn_sink;
 } mla_weights_desc;
 
 typedef struct mla_handle mla_handle;
@@ -301,6 +308,31 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos,
                 const float* sin, void* out, void* head_out, void* kv_cache,
                 int n_blocks, const int32_t* slot_mapping, void* ws, size_t ws_bytes,
                 void* stream);
+
+/* ---- DeepSeek-V4 QKV projection ---------------------------------------------------- */
+
+/* The DeepSeek-V4 form of the QKV projection ("QKV CTE MLA Kernel API
+ * Reference", qkv_mla_mx_deepseek_v4), on the handle's [wq_a | wkv_a] (the
+ * fused first projection wqkv [D, r_q + kv_dim], kv_dim = r_kv + d_r),
+ * q_norm_w and wq_b (wkv_b and wo are not used):
+ *   qr, kv = split(x @ wqkv)
+ *   q      = RMSNorm(qr, q_norm_w) @ wq_b, viewed [S, H, hd] (hd = d_n + d_r)
+ *   q_h    = q_h / sqrt(mean(q_h^2) + norm_eps)       (per head, no gain)
+ *   q_h[hd - d_r:]   rotated by interleaved RoPE at the token's position
+ *   kv     = RMSNorm(kv, kv_norm_w) over all kv_dim columns
+ *   kv[kv_dim - d_r:] rotated by interleaved RoPE
+ * for S tokens with their own cos/sin rows (any positions).
+ * hidden     device [S, D] act dtype; cos, sin device [S, d_r/2] fp32
+ * kv_norm_w  device [r_kv + d_r] fp32 (the V4 kv gamma covers the whole row)
+ * q_out      device [S, H, hd] act dtype; kv_out device [S, r_kv + d_r] act
+ *            dtype ([latent | rotated tail], the form of a cache row)
+ * ws         device workspace of mla_workspace_bytes(h, S, 1)
+ * Needs q_lora_rank > 0 (MLA_ERR_UNSUPPORTED otherwise). Readings where the
+ * page is brief: the per-head norm is the RMS form with norm_eps; RoPE is the
+ * interleaved pairing of the decode kernel. */
+int mla_v4_qkv(mla_handle* h, const void* hidden, int S, const float* cos, const float* sin,
+               const float* kv_norm_w, void* q_out, void* kv_out, void* ws, size_t ws_bytes,
+               void* stream);
 
 /* ---- misc ------------------------------------------------------------------------ */
 

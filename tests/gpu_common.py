@@ -80,10 +80,12 @@ class DecodeCase:
     """A decode step on the GPU and its inputs, for one workload."""
 
     def __init__(self, workload, batch=None, ctx=None, row_layout=ref.LATENT_FIRST, device="cuda",
-                 input_norm_w=None, inv_freq=None):
-        """input_norm_w [hidden] / inv_freq [qk_rope/2]: optional fp32 numpy arrays for
-        this step's input RMSNorm and RoPE frequency table (both sides get the same values)."""
+                 input_norm_w=None, inv_freq=None, attn_sink=None):
+        """input_norm_w [hidden] / inv_freq [qk_rope/2] / attn_sink [n_heads]: optional fp32
+        numpy arrays for this step's input RMSNorm, RoPE frequency table and per-head sink
+        logits (both sides get the same values)."""
         ensure_built()
+        self.attn_sink = None if attn_sink is None else np.asarray(attn_sink, np.float32)
         self.input_norm_w = None if input_norm_w is None else np.asarray(input_norm_w, np.float32)
         self.inv_freq = None if inv_freq is None else np.asarray(inv_freq, np.float32)
         self.w = workload
@@ -91,7 +93,7 @@ class DecodeCase:
         self.row_layout = row_layout
         self.weights = wl.make_weights(s, workload.seed)
         self.inp = wl.make_decode_inputs(workload, batch=batch, ctx=ctx)
-        self.layer = MlaLayer(s, self.weights, row_layout=row_layout, device=device)
+        self.layer = MlaLayer(s, self.weights, row_layout=row_layout, device=device, attn_sink=self.attn_sink)
         self.act = ACT_TORCH[s.act_dtype]
         self.device = device
         inp = self.inp
@@ -152,6 +154,6 @@ class DecodeCase:
         q_abs, q_pe, new_cache = ref.decode_qkv(s, W, inp.hidden[seqs], cos, sin, cache, slots,
                                                 self.row_layout, input_norm_w=self.input_norm_w)
         out, head_out = ref.decode_attn(s, W, q_abs, q_pe, new_cache, table,
-                                        inp.context_lens[seqs], self.row_layout)
+                                        inp.context_lens[seqs], self.row_layout, attn_sink=self.attn_sink)
         return dict(q_abs=q_abs, q_pe=q_pe, cache=new_cache, out=out, head_out=head_out,
                     slots=slots, blocks=blocks, seqs=seqs)

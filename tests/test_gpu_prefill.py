@@ -20,12 +20,13 @@ V2LITE_PREFILL = dataclasses.replace(wl.WORKLOADS["v3_prefill_bf16"], shape=wl.V
 V3_FP8_PREFILL = dataclasses.replace(wl.WORKLOADS["v3_prefill_bf16"], shape=wl.WORKLOADS["v3_fp8"].shape, seed=12)
 
 
-def run_prefill(workload, S, rows=None, with_cache=False):
+def run_prefill(workload, S, rows=None, with_cache=False, attn_sink=None):
+    """attn_sink: optional fp32 [n_heads] sink logits, given to both sides."""
     ensure_built()
     s = workload.shape
     weights = wl.make_weights(s, workload.seed)
     x, pos = wl.make_prefill_inputs(workload, seq_len=S)
-    layer = MlaLayer(s, weights)
+    layer = MlaLayer(s, weights, attn_sink=attn_sink)
     act = ACT_TORCH[s.act_dtype]
     xd = to_dev(x, act)
     cos, sin = layer.rope(torch.from_numpy(pos).cuda())
@@ -41,7 +42,7 @@ def run_prefill(workload, S, rows=None, with_cache=False):
     torch.cuda.synchronize()
     W = ref.weights_fp64(weights)
     rcos, rsin = ref.rope_cos_sin(pos, s.qk_rope, s.rope_theta)
-    r_out, r_head, r_rows = ref.prefill(s, W, x, rcos, rsin, rows=rows)
+    r_out, r_head, r_rows = ref.prefill(s, W, x, rcos, rsin, rows=rows, attn_sink=attn_sink)
     sel = np.arange(S) if rows is None else np.asarray(rows)
     tol = TOL[s.act_dtype]
     assert_close_per_head(to_np(head)[sel], r_head, tol, "head_out")
