@@ -5,8 +5,9 @@
 
 A step is one pass of the hot path over one synthetic batch: for decode
 workloads mla_decode_qkv + mla_decode_attn (front-fold, scatter, absorbed
-attention, V extraction, o_proj) for `batch` tokens; for the prefill workload
-one mla_prefill of the whole sequence. Inputs are resident in HBM when the
+attention, V extraction, o_proj) for `batch` tokens; for the prefill workloads
+one mla_prefill of the whole sequence; for v4_qkv_bf16 one mla_v4_qkv (the
+DeepSeek-V4 QKV projection) of 8192 tokens. Inputs are resident in HBM when the
 timed region starts; the step is replayed from a CUDA graph; L2 is flushed
 (256 MiB write, outside the timed events) before every timed step. `e2e`
 times the same step through the C-ABI from pinned host buffers with the
@@ -43,6 +44,7 @@ from head_latent_attention_decode_b200 import workloads as wl  # noqa: E402
 DEFAULT_WORKLOAD = "v2lite_bf16"
 METRIC_DECODE = "MLA decode tokens/s (one layer step: front-fold + absorbed paged attention + o_proj)"
 METRIC_PREFILL = "MLA prefill TFLOP/s (causal expanded path)"
+METRIC_V4 = "MLA DeepSeek-V4 QKV projection TFLOP/s"
 
 
 # ---------------------------------------------------------------------------
@@ -86,6 +88,12 @@ def prefill_flops(s: wl.MlaShape, S: int) -> dict:
     return dict(total=proj + attn + oproj, attn=attn)
 
 
+def v4_flops(s: wl.MlaShape, S: int) -> dict:
+    """x @ [wq_a | wkv_a] and qn @ wq_b (the two GEMMs of the V4 projection)."""
+    qb = 2 * S * s.q_lora_rank * s.n_heads * (s.qk_nope + s.qk_rope)
+    return dict(total=2 * S * s.hidden * (s.q_lora_rank + s.kv_row_dim) + qb, qb=qb)
+
+
 # ---------------------------------------------------------------------------
 # DRAM traffic of the dominant kernel, from the committed ncu summary
 # ---------------------------------------------------------------------------
@@ -94,12 +102,15 @@ KERNEL_SOURCES = {
     "tc_attn_decode_kernel": "tc_attn.cuh",
     "tc_attn_pair_kernel": "tc_attn_pair.cuh",
     "tc_prefill_attn_kernel": "tc_prefill_attn.cuh",
+    "tc_gemm_kernel": "tc_gemm.cuh",
 }
 
 
 def dominant_kernel(w: wl.Workload) -> str:
     if w.mode == "prefill":
         return "tc_prefill_attn_kernel"
+    if w.mode == "v4qkv":
+        return "tc_gemm_kernel"
     return "tc_attn_pair_kernel" if w.shape.n_heads <= 32 else "tc_attn_decode_kernel"
 
 
@@ -311,6 +322,50 @@ class PrefillStep:
         self.h_out.copy_(self.out, non_blocking=True)
 
 
+class V4QkvStep:
+    def __init__(self, w: wl.Workload, rank: int):
+        from head_latent_attention_decode_b200.layer import MlaLayer
+        self.w = w
+        s = self.s = w.shape
+        self.weights = wl.make_weights(s, w.seed)
+        x, pos = wl.make_prefill_inputs(w, seed_offset=200 + 1000 * rank)
+        self.layer = layer = MlaLayer(s, self.weights)
+        self.S = S = x.shape[0]
+        self.hidden = torch.from_numpy(x).to(layer.act).cuda()
+        self.positions = torch.from_numpy(pos).cuda()
+        self.cos, self.sin = layer.rope(self.positions)
+        g = 1.0 + np.random.default_rng(w.seed + 300).uniform(-0.3, 0.3, s.kv_row_dim)
+        self.kv_w = torch.from_numpy(g.astype(np.float32)).cuda()
+        self.q = torch.empty((S, s.n_heads, s.qk_nope + s.qk_rope), dtype=layer.act, device="cuda")
+        self.kv = torch.empty((S, s.kv_row_dim), dtype=layer.act, device="cuda")
+        self.ws = layer.workspace(S, 1)
+        self.flops = v4_flops(s, S)
+        self.tokens = S
+
+    def run(self):
+        mla.mla_v4_qkv(self.layer.handle, self.hidden, self.cos, self.sin, self.kv_w, self.q, self.kv, self.ws)
+
+    def e2e_setup(self):
+        self.h_hidden = self.hidden.cpu().pin_memory()
+        self.h_pos = self.positions.cpu().pin_memory()
+        self.h_q = torch.empty(self.q.shape, dtype=self.q.dtype).pin_memory()
+        self.h_kv = torch.empty(self.kv.shape, dtype=self.kv.dtype).pin_memory()
+        self.d_hidden, self.d_pos = torch.empty_like(self.hidden), torch.empty_like(self.positions)
+        return (self.h_hidden.numel() * self.h_hidden.element_size() + self.h_pos.numel() * 4,
+                self.h_q.numel() * self.h_q.element_size() + self.h_kv.numel() * self.h_kv.element_size())
+
+    def run_e2e(self):
+        self.d_hidden.copy_(self.h_hidden, non_blocking=True)
+        self.d_pos.copy_(self.h_pos, non_blocking=True)
+        s = self.s
+        cos = torch.empty((self.S, s.qk_rope // 2), dtype=torch.float32, device="cuda")
+        sin = torch.empty_like(cos)
+        mla.mla_rope_cos_sin(self.d_pos, s.qk_rope, s.rope_theta, cos, sin)
+        mla.mla_v4_qkv(self.layer.handle, self.d_hidden, cos, sin, self.kv_w, self.q, self.kv, self.ws)
+        self.h_q.copy_(self.q, non_blocking=True)
+        self.h_kv.copy_(self.kv, non_blocking=True)
+
+
 def capture(step, stream):
     """CUDA graph of one step (and the number of library launches in it)."""
     g = torch.cuda.CUDAGraph()
@@ -366,6 +421,21 @@ def cpu_oracle_sample(w: wl.Workload, budget_s: float = 12.0, max_reps: int = 10
     weights = wl.make_weights(s, w.seed)
     W = ref.weights_fp64(weights)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    if w.mode == "v4qkv":
+        # the oracle on a block of tokens, repeated within the budget
+        x, pos = wl.make_prefill_inputs(w, seq_len=64)
+        g = 1.0 + np.random.default_rng(w.seed + 300).uniform(-0.3, 0.3, s.kv_row_dim)
+        cos, sin = ref.rope_cos_sin(pos, s.qk_rope, s.rope_theta)
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            ref.v4_qkv(s, W, x, cos, sin, g)
+            reps += 1
+            dt = time.perf_counter() - t0
+            if dt >= budget_s or reps >= max_reps:
+                break
+        f = v4_flops(s, len(x))["total"] * reps
+        return dict(value=f / dt / 1e12, unit="TFLOP/s", cores=threads, kind="oracle",
+                    sample=f"{len(x)} of {w.seq_len} tokens, {reps} oracle passes in {dt:.1f} s", seconds=dt)
     if w.mode == "prefill":
         S = w.seq_len
         x, pos = wl.make_prefill_inputs(w)
@@ -412,7 +482,7 @@ def run_ours(args, world, rank, local):
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
     tc_peak = peaks.get("bf16_tflops", 1590.0)
     peak_src = "measured" if peaks else "fallback"
-    step = DecodeStep(w, rank) if w.mode == "decode" else PrefillStep(w, rank)
+    step = {"decode": DecodeStep, "prefill": PrefillStep, "v4qkv": V4QkvStep}[w.mode](w, rank)
     stream = torch.cuda.Stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     torch.cuda.synchronize()
@@ -437,7 +507,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         ms = all_max(float(np.mean(times)), world)
         # dominant kernel, timed live with event nodes around its launch
-        kname = "attn" if w.mode == "decode" else "prefill_attn"
+        kname = {"decode": "attn", "prefill": "prefill_attn", "v4qkv": "v4_qb"}[w.mode]
         kms = all_max(kernel_time(step, kname, max(3, args.steps), flush, stream), world)
         kern = dominant_kernel(w) if torch.cuda.get_device_capability()[0] == 10 else kname
         # end to end through the C-ABI with host buffers
@@ -473,6 +543,18 @@ def run_ours(args, world, rank, local):
         e2e_val = toks / (e2e / 1e3)
         metric = METRIC_DECODE
         cfg = workload_config(w, world, step.inp.context_lens)
+    elif w.mode == "v4qkv":
+        fl = step.flops
+        value, unit = fl["total"] * world / (ms / 1e3) / 1e12, "TFLOP/s"
+        achieved = fl["qb"] / (kms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": kern, "achieved": round(achieved, 2),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                "peak_source": peak_src, "kernel_ms": round(kms, 4),
+                "algorithmic_flops": fl["qb"], "traffic": measured_traffic(kern, w.name)}
+        extra = {"tokens_per_s": round(toks / (ms / 1e3), 1), "step_flops": fl["total"]}
+        e2e_val = fl["total"] * world / (e2e / 1e3) / 1e12
+        metric = METRIC_V4
+        cfg = workload_config(w, world)
     else:
         fl = step.flops
         value, unit = fl["total"] * world / (ms / 1e3) / 1e12, "TFLOP/s"
@@ -508,7 +590,7 @@ def workload_config(w: wl.Workload, world: int, context_lens=None) -> dict:
     """The `config` object of a bench line (both arms)."""
     s = w.shape
     l2 = "flushed before each timed step (256 MiB write, outside the events)"
-    if w.mode == "prefill":
+    if w.mode in ("prefill", "v4qkv"):
         return {"workload": w.name, "seq_len": w.seq_len, "batch": 1, "weights": s.weight_dtype, "heads": s.n_heads,
                 "hidden": s.hidden, "l2": l2, "parallelism": f"replicas x{world}"}
     if context_lens is None:
@@ -534,7 +616,7 @@ def run_reference(args, world, rank):
     v = float(np.mean(vals))
     cb["value"] = v
     cb["sample"] = cb["sample"] + f"; {args.steps} bench steps, each one oracle pass (set-up excluded)"
-    line = {"impl": "reference", "metric": METRIC_DECODE if w.mode == "decode" else METRIC_PREFILL,
+    line = {"impl": "reference", "metric": {"decode": METRIC_DECODE, "prefill": METRIC_PREFILL, "v4qkv": METRIC_V4}[w.mode],
             "value": round(v, 4), "unit": cb["unit"], "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(float(np.mean(secs)) * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

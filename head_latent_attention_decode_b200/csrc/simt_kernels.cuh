@@ -235,6 +235,62 @@ __global__ void __launch_bounds__(256) q_headnorm_rope_kernel(T* q, long long ld
   }
 }
 
+// The same for bf16 heads with hd and d_r multiples of 8 and 16-byte aligned
+// rows: 8 lanes per head, each moving 16-byte chunks (chunk c of the head on
+// lane c % 8), so a warp streams four heads with full 128-byte accesses.
+// grid (n, ceil(H / 32)), 256 threads; hd <= 512.
+__global__ void __launch_bounds__(256) q_headnorm_rope_bf16x8_kernel(bf16* q, long long ldq, int H, int hd, int d_r,
+                                                                     const float* cos, const float* sin, float eps) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int t = blockIdx.x, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * 32 + (threadIdx.x >> 3);   // 4 heads per warp, 8 lanes per head
+  const int i = lane & 7;
+  const int nc = hd / 8, base = hd - d_r, half = d_r / 2;
+  uint4* qh = reinterpret_cast<uint4*>(q + (long long)t * ldq + (long long)(h < H ? h : 0) * hd);
+  uint4 v[8];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int c = i + 8 * k;
+    v[k] = (h < H && c < nc) ? qh[c] : make_uint4(0, 0, 0, 0);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(p2[j]);
+      ss += f.x * f.x + f.y * f.y;
+    }
+  }
+  // the head's sum over its 8 lanes (the xor partners stay inside the group)
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+  if (h >= H) return;
+  const float r = rsqrtf(ss / (float)hd + eps);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int c = i + 8 * k;
+    if (c >= nc) break;
+    __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&v[k]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __bfloat1622float2(p2[j]);
+      f.x *= r;
+      f.y *= r;
+      const int e = 8 * c + 2 * j;   // even element index within the head
+      if (e >= base) {
+        const int pi = (e - base) / 2;
+        float o0, o1;
+        rope_pair(f.x, f.y, cos[(long long)t * half + pi], sin[(long long)t * half + pi], &o0, &o1);
+        f.x = o0;
+        f.y = o1;
+      }
+      p2[j] = __floats2bfloat162_rn(f.x, f.y);
+    }
+    qh[c] = v[k];
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Absorbed split-KV decode attention (CUDA cores). grid (n_splits, n, head
 // groups of 8), 256 threads: warp w owns head g*8 + w; lane = cache row of the

@@ -822,9 +822,17 @@ static inline int tc_v4_qkv(const mla_handle* h, const void* hidden, int S, cons
   CUtensorMap bq;
   if ((st = prefill_weight_map(h, &bq, T.b_Wqb, L.Wqb, L.sWqb, L.Hq, rq, 0, L.Hq, dq, true, s)) != MLA_OK) return st;
   g2.static_op = sop;
-  if ((st = launch_gemm(mq, bq, g2, 256, 1, T.num_sms, s)) != MLA_OK) return st;
-  launch_pdl(q_headnorm_rope_kernel<bf16>, S, 256, 0, s, (bf16*)q_out, (long long)L.Hq, H, dn + dr, dr, cos, sin,
-             c.norm_eps);
+  mla_timer_begin("v4_qb", s);
+  st = launch_gemm(mq, bq, g2, 256, 1, T.num_sms, s);
+  mla_timer_end("v4_qb", s);
+  if (st != MLA_OK) return st;
+  const int hd = dn + dr;
+  if (hd % 8 == 0 && dr % 8 == 0 && hd <= 512 && ((uintptr_t)q_out & 15) == 0)
+    launch_pdl(q_headnorm_rope_bf16x8_kernel, dim3(S, (unsigned)cdiv(H, 32)), 256, 0, s, (bf16*)q_out,
+               (long long)L.Hq, H, hd, dr, cos, sin, c.norm_eps);
+  else
+    launch_pdl(q_headnorm_rope_kernel<bf16>, S, 256, 0, s, (bf16*)q_out, (long long)L.Hq, H, hd, dr, cos, sin,
+               c.norm_eps);
   mla_count_launch(1);
   return MLA_OK;
 }

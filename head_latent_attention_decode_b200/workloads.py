@@ -62,7 +62,7 @@ class MlaShape:
 class Workload:
     name: str
     shape: MlaShape
-    mode: str                  # "decode" | "prefill"
+    mode: str                  # "decode" | "prefill" | "v4qkv" (the DeepSeek-V4 QKV projection)
     batch: int                 # decode tokens (one per sequence); 1 for prefill
     ctx_lo: int                # context length range (inclusive) per sequence
     ctx_hi: int
@@ -107,6 +107,11 @@ WORKLOADS = {
         "v3_prefill_fp8", V3_FP8, "prefill", batch=1, ctx_lo=0, ctx_hi=0, cache_fill="none",
         seed=6, seq_len=8192, description="DeepSeek-V3-shaped MLA prefill, FP8-E4M3 weights with "
         "128x128 fp32 block scales, bf16 activations, seq 8192 causal, expanded K/V"),
+    "v4_qkv_bf16": Workload(
+        "v4_qkv_bf16", V3, "v4qkv", batch=1, ctx_lo=0, ctx_hi=0, cache_fill="none",
+        seed=7, seq_len=8192, description="DeepSeek-V4 form of the QKV projection on "
+        "DeepSeek-V3-sized matrices (hidden 7168, q_lora 1536, kv_dim 576, 128 heads of "
+        "192), bf16, 8192 tokens"),
 }
 
 

@@ -348,7 +348,8 @@ uint64_t mla_kernel_launch_count(void);
  * "attn" (decode attention), "prefill_attn", and the decode weight GEMMs
  * "gemm_w1" (down-projection), "gemm_qb" (wq_b), "gemm_uk" (absorption),
  * "gemm_uv" (V extraction), "gemm_o" (o_proj), each including the operand
- * conversion or weight dequantisation it launches. NULL clears the timer. Inside a
+ * conversion or weight dequantisation it launches, and "v4_qb" (the wq_b GEMM
+ * of mla_v4_qkv on tensor cores). NULL clears the timer. Inside a
  * stream capture the records become external event-record nodes of the graph.
  * Process-wide; not thread-safe against concurrent launches. */
 int mla_set_kernel_timer(const char* kernel, void* start_event, void* stop_event);
