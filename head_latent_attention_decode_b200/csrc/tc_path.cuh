@@ -212,24 +212,18 @@ struct FrontFoldTcArgs {
   bf16* qn; bf16* q_nope; bf16* q_pe;
   bf16* cache; long long n_rows; const int* slot; int layout;
   int* flag;
+  int q_cols;   // columns of the q part per CTA: all r_q, or whole heads of d_n + d_r
 };
 
-// One CTA per token: sum the K-split partials of x @ W1, then
-//   q latent -> RMSNorm * q_norm_w -> qn (bf16)                          (r_q > 0)
-//   or q -> q_nope (bf16) and RoPE(q_pe) (bf16)                          (r_q = 0)
-//   kv latent -> RMSNorm * kv_norm_w, k_pe -> RoPE, row -> cache[slot]
-__global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
-  griddep_wait();
-  griddep_launch_dependents();
-  extern __shared__ float y[];   // [N1]
-  __shared__ float red[32];
-  const int t = blockIdx.x;
-  const float* yp = p.Yp + (long long)t * p.N1;
-  if (p.N1 % 4 == 0 && p.split_stride % 4 == 0 && ((uintptr_t)p.Yp & 15) == 0) {
-    // 16-byte loads, the first eight splits' loads all in flight before the sum
+// Sum the K-split partials of columns [c0, c0 + w) of token t's row of x @ W1
+// into y[0, w) (16-byte loads when aligned, the first eight splits' loads all
+// in flight before the sum).
+__device__ __forceinline__ void frontfold_sum(const FrontFoldTcArgs& p, int t, int c0, int w, float* y) {
+  const float* yp = p.Yp + (long long)t * p.N1 + c0;
+  if (w % 4 == 0 && c0 % 4 == 0 && p.N1 % 4 == 0 && p.split_stride % 4 == 0 && ((uintptr_t)p.Yp & 15) == 0) {
     const float4* yp4 = reinterpret_cast<const float4*>(yp);
     const long long st4 = p.split_stride >> 2;
-    for (int c = threadIdx.x; c < (p.N1 >> 2); c += blockDim.x) {
+    for (int c = threadIdx.x; c < (w >> 2); c += blockDim.x) {
       float4 v[8];
 #pragma unroll
       for (int s = 0; s < 8; ++s) v[s] = s < p.splits ? yp4[s * st4 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -237,42 +231,65 @@ __global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
 #pragma unroll
       for (int s = 1; s < 8; ++s) { acc.x += v[s].x; acc.y += v[s].y; acc.z += v[s].z; acc.w += v[s].w; }
       for (int s = 8; s < p.splits; ++s) {
-        const float4 w = yp4[s * st4 + c];
-        acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
+        const float4 u = yp4[s * st4 + c];
+        acc.x += u.x; acc.y += u.y; acc.z += u.z; acc.w += u.w;
       }
       reinterpret_cast<float4*>(y)[c] = acc;
     }
   } else {
-    for (int c = threadIdx.x; c < p.N1; c += blockDim.x) {
+    for (int c = threadIdx.x; c < w; c += blockDim.x) {
       float acc = 0.f;
       for (int s = 0; s < p.splits; ++s) acc += yp[s * p.split_stride + c];
       y[c] = acc;
     }
   }
-  __syncthreads();
+}
+
+// grid (tokens, 1 + q slices). For token t, CTA 0 sums the kv part of the
+// K-split partials of x @ W1 and does
+//   kv latent -> RMSNorm * kv_norm_w, k_pe -> RoPE, row -> cache[slot];
+// CTA g >= 1 sums its slice of the q part and does
+//   q latent -> RMSNorm * q_norm_w -> qn (bf16)            (r_q > 0: one slice, all r_q)
+//   or q -> q_nope (bf16) and RoPE(q_pe) (bf16)            (r_q = 0: slices of whole heads)
+__global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  extern __shared__ float y[];   // [max(q_cols, r_kv + d_r)]
+  __shared__ float red[32];
+  const int t = blockIdx.x, g = blockIdx.y;
   const int half = p.dr / 2;
-  if (p.rq) {
-    float ss = 0.f;
-    for (int i = threadIdx.x; i < p.rq; i += blockDim.x) ss += y[i] * y[i];
-    const float r = rsqrtf(block_sum(ss, red) / (float)p.rq + p.eps);
-    for (int i = threadIdx.x; i < p.rq; i += blockDim.x)
-      p.qn[(long long)t * p.rq + i] = __float2bfloat16_rn(y[i] * r * p.q_norm_w[i]);
-  } else {
-    const int hd = p.dn + p.dr;
-    for (int idx = threadIdx.x; idx < p.H * p.dn; idx += blockDim.x) {
-      const int h = idx / p.dn, j = idx % p.dn;
-      p.q_nope[(long long)t * p.H * p.dn + idx] = __float2bfloat16_rn(y[h * hd + j]);
+  if (g > 0) {
+    const int c0 = (g - 1) * p.q_cols;
+    const int w = min(p.Nq1, c0 + p.q_cols) - c0;
+    if (w <= 0) return;
+    frontfold_sum(p, t, c0, w, y);
+    __syncthreads();
+    if (p.rq) {
+      float ss = 0.f;
+      for (int i = threadIdx.x; i < p.rq; i += blockDim.x) ss += y[i] * y[i];
+      const float r = rsqrtf(block_sum(ss, red) / (float)p.rq + p.eps);
+      for (int i = threadIdx.x; i < p.rq; i += blockDim.x)
+        p.qn[(long long)t * p.rq + i] = __float2bfloat16_rn(y[i] * r * p.q_norm_w[i]);
+    } else {
+      const int hd = p.dn + p.dr, h0 = c0 / hd, nh = w / hd;
+      for (int idx = threadIdx.x; idx < nh * p.dn; idx += blockDim.x) {
+        const int h = idx / p.dn, j = idx % p.dn;
+        p.q_nope[((long long)t * p.H + h0 + h) * p.dn + j] = __float2bfloat16_rn(y[h * hd + j]);
+      }
+      for (int idx = threadIdx.x; idx < nh * half; idx += blockDim.x) {
+        const int h = idx / half, i = idx % half;
+        float o0, o1;
+        rope_pair(y[h * hd + p.dn + 2 * i], y[h * hd + p.dn + 2 * i + 1], p.cos[(long long)t * half + i],
+                  p.sin[(long long)t * half + i], &o0, &o1);
+        p.q_pe[((long long)t * p.H + h0 + h) * p.dr + 2 * i] = __float2bfloat16_rn(o0);
+        p.q_pe[((long long)t * p.H + h0 + h) * p.dr + 2 * i + 1] = __float2bfloat16_rn(o1);
+      }
     }
-    for (int idx = threadIdx.x; idx < p.H * half; idx += blockDim.x) {
-      const int h = idx / half, i = idx % half;
-      float o0, o1;
-      rope_pair(y[h * hd + p.dn + 2 * i], y[h * hd + p.dn + 2 * i + 1], p.cos[(long long)t * half + i],
-                p.sin[(long long)t * half + i], &o0, &o1);
-      p.q_pe[((long long)t * p.H + h) * p.dr + 2 * i] = __float2bfloat16_rn(o0);
-      p.q_pe[((long long)t * p.H + h) * p.dr + 2 * i + 1] = __float2bfloat16_rn(o1);
-    }
+    return;
   }
-  const float* kv = y + p.Nq1;
+  frontfold_sum(p, t, p.Nq1, p.rkv + p.dr, y);
+  __syncthreads();
+  const float* kv = y;
   float ss = 0.f;
   for (int i = threadIdx.x; i < p.rkv; i += blockDim.x) ss += kv[i] * kv[i];
   const float r = rsqrtf(block_sum(ss, red) / (float)p.rkv + p.eps);
@@ -610,9 +627,14 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   f.qn = (bf16*)(tw + W.qn); f.q_nope = (bf16*)(tw + W.q_nope); f.q_pe = (bf16*)q_pe;
   f.cache = (bf16*)kv_cache; f.n_rows = (long long)n_blocks * c.block_size; f.slot = slot_mapping;
   f.layout = c.row_layout; f.flag = flag;
-  const size_t ff_smem = (size_t)L.N1 * 4;
+  // the q part in slices: all of r_q (its RMSNorm spans it), or about a third
+  // of the heads each without q_lora; the kv part in CTA 0
+  const int hd = dn + dr;
+  f.q_cols = rq ? rq : (int)cdiv(H, 3) * hd;
+  const int q_slices = (int)cdiv(L.Nq1, f.q_cols);
+  const size_t ff_smem = (size_t)(f.q_cols > L.R ? f.q_cols : L.R) * 4;
   if (ff_smem > 48 * 1024) cudaFuncSetAttribute(frontfold_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ff_smem);
-  launch_pdl(frontfold_tc_kernel, n, 512, ff_smem, s, f);
+  launch_pdl(frontfold_tc_kernel, dim3(n, 1 + q_slices), 512, ff_smem, s, f);
   mla_count_launch(1);
   // 3. q = qn @ wq_b with q_nope out and RoPE(q_pe) out (swap-AB)
   if (rq) {
