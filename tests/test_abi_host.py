@@ -119,6 +119,20 @@ def test_calls_reject_null_handle_and_bad_sizes(lib):
     v = ctypes.c_int()
     assert lib.mla_read_device_flag(None, ctypes.byref(v), None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_clear_device_flag(None, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_v4_qkv(None, P, 1, P, P, P, P, P, P, 1 << 20, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_v4_qkv(None, P, -1, P, P, P, P, P, P, 1 << 20, None) == mla.MLA_ERR_INVALID_ARG
+
+
+def test_weights_descriptor_ends_with_the_sink():
+    """The C struct's field order: twelve weight / gamma / scale pointers, then
+    the optional attn_sink pointer (a zero-initialised descriptor has no sink)."""
+    names = [f[0] for f in mla.mla_weights_desc._fields_]
+    assert names[-1] == "attn_sink" and len(names) == 13
+    assert ctypes.sizeof(mla.mla_weights_desc) == 13 * ctypes.sizeof(ctypes.c_void_p)
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "mla.h")).read()
+    body = hdr[hdr.index("typedef struct {\n  const void* wq_a;"):hdr.index("} mla_weights_desc;")]
+    fields = [ln.strip().rstrip(";").split()[-1].lstrip("*") for ln in body.splitlines()[1:] if ln.strip()]
+    assert fields == names
 
 
 def test_launch_counter_starts_at_zero_without_gpu_work(lib):
