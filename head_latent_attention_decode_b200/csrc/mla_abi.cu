@@ -133,7 +133,7 @@ static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
   W.qn = put((size_t)n * (c->q_lora_rank ? c->q_lora_rank : 1) * a);
   W.Q = put((size_t)n * L.Hq * 4);
   W.part_o = put((size_t)n * W.splits * H * rkv * 4);
-  W.part_ml = put((size_t)n * W.splits * H * 2 * 4);
+  W.part_ml = put((size_t)n * W.splits * H * 2 * 4 * 2);   // one (m, l) copy per CTA of a pair
   W.o_lat = put((size_t)n * H * rkv * a);
   W.head = put((size_t)n * H * dv * a);
   W.xn = put((size_t)n * c->hidden * a);
@@ -495,8 +495,8 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
     count_launch();
     dim3 cg(n, H);
     const float* sink = h->has_sink ? (const float*)(h->base + L.sink) : nullptr;
-    if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat, sink);
-    else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat, sink);
+    if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat, sink, 0, 0);
+    else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat, sink, 0, 0);
     count_launch();
   }
   // head_out[h] = o_lat[h] @ W_UV[h]

@@ -402,51 +402,58 @@ __global__ void __launch_bounds__(256) attn_decode_simt_kernel(AttnArgs p) {
 // Merge split partials: o_lat = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s.
 // With a per-head sink logit z_h ("Struct MlaWeights", attn_sink) the softmax
 // has one more column that carries no value: M also covers z_h and the
-// denominator gains e^{z_h - M}. grid (n, H), 128 threads x 4 consecutive
-// columns (r_kv <= 512, r_kv % 4 == 0). Writes o_lat [n, H, r_kv] in act dtype.
+// denominator gains e^{z_h - M}. Kernels that split the latent columns over a
+// CTA pair store one (m, l) copy per CTA: columns c >= half_cols then use the
+// copy ml_r floats further on (half_cols = 0: one copy for all columns).
+// grid (n, H), 128 threads x 4 consecutive columns (r_kv <= 512, r_kv % 4 == 0).
+// Writes o_lat [n, H, r_kv] in act dtype.
 template <typename T>
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, const float* part_ml, int n_splits,
-                                                           int H, int r_kv, T* o_lat, const float* sink) {
+                                                           int H, int r_kv, T* o_lat, const float* sink,
+                                                           long long ml_r, int half_cols) {
   griddep_wait();
   griddep_launch_dependents();
-  __shared__ float wsh[64];
-  __shared__ float inv_sh;
+  __shared__ float wsh[2][64];
+  __shared__ float inv_sh[2];
   const int t = blockIdx.x, h = blockIdx.y;
-  if (threadIdx.x < 32) {
+  const int warp = threadIdx.x >> 5;
+  if (warp < (half_cols > 0 ? 2 : 1)) {   // warp w: the weights of stats copy w
+    const float* ml = part_ml + warp * ml_r;
     float M = -INFINITY;
-    for (int s = threadIdx.x; s < n_splits; s += 32) {
+    for (int s = threadIdx.x & 31; s < n_splits; s += 32) {
       const long long base = ((long long)t * n_splits + s) * H + h;
-      if (part_ml[base * 2 + 1] > 0.f) M = fmaxf(M, part_ml[base * 2]);
+      if (ml[base * 2 + 1] > 0.f) M = fmaxf(M, ml[base * 2]);
     }
     M = warp_max(M);
     const float z = sink ? sink[h] : -INFINITY;
     M = fmaxf(M, z);
-    float den = (threadIdx.x == 0 && z > -INFINITY) ? __expf(z - M) : 0.f;
-    for (int s = threadIdx.x; s < n_splits; s += 32) {
+    float den = ((threadIdx.x & 31) == 0 && z > -INFINITY) ? __expf(z - M) : 0.f;
+    for (int s = threadIdx.x & 31; s < n_splits; s += 32) {
       const long long base = ((long long)t * n_splits + s) * H + h;
-      const float l = part_ml[base * 2 + 1];
-      const float w = (l > 0.f) ? __expf(part_ml[base * 2] - M) : 0.f;
-      if (s < 64) wsh[s] = w;
+      const float l = ml[base * 2 + 1];
+      const float w = (l > 0.f) ? __expf(ml[base * 2] - M) : 0.f;
+      if (s < 64) wsh[warp][s] = w;
       den += w * l;
     }
     den = warp_sum(den);
-    if (threadIdx.x == 0) inv_sh = den > 0.f ? 1.f / den : 0.f;
+    if ((threadIdx.x & 31) == 0) inv_sh[warp] = den > 0.f ? 1.f / den : 0.f;
   }
   __syncthreads();
   const int c = threadIdx.x * 4;
   if (c >= r_kv) return;
+  const int cp = (half_cols > 0 && c >= half_cols) ? 1 : 0;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   const int ns = n_splits < 64 ? n_splits : 64;
 #pragma unroll 4
   for (int s = 0; s < ns; ++s) {
-    const float w = wsh[s];
+    const float w = wsh[cp][s];
     if (w == 0.f) continue;
     const long long base = ((long long)t * n_splits + s) * H + h;
     const float4 v = *reinterpret_cast<const float4*>(part_o + base * r_kv + c);
     acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
     acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
   }
-  const float inv = inv_sh;
+  const float inv = inv_sh[cp];
   T* o = o_lat + ((long long)t * H + h) * r_kv + c;
   o[0] = from_f32<T>(acc.x * inv); o[1] = from_f32<T>(acc.y * inv);
   o[2] = from_f32<T>(acc.z * inv); o[3] = from_f32<T>(acc.w * inv);

@@ -39,8 +39,12 @@ struct TcAttnArgs {
   int lat_col0, rope_col0;
   float scale_log2;
   float* part_o;   // [n, splits, H, 512]
-  float* part_ml;  // [n, splits, H, 2]
+  float* part_ml;  // [n, splits, H, 2], and the same again at part_ml + ml_r
   int* flag;
+  // CTA r of a pair stores its own (m, l) at part_ml + r * ml_r: the two CTAs
+  // add the same two partial scores in a different rounding (own fp32 + peer
+  // f16), so each half of the latent is normalised with its own statistics
+  long long ml_r;
   // optional tracing: %globaltimer stamps of cluster 0, both CTAs, for the
   // first 64 tiles, [CTA][tile][32]: softmax (head 0) 0 iteration start,
   // 2 peer partial arrived, 6 S ready, 7 S read, 11 partials added, 3 peer
@@ -109,10 +113,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   const int r0 = sp * a.chunk, r1 = min(L, r0 + a.chunk);
   const int T = r1 > r0 ? (r1 - r0 + 63) / 64 : 0;
   const long long unit = (long long)b * a.splits + sp;
+  float* const ml = a.part_ml + r * a.ml_r;   // this CTA's (m, l) copy
   if (T == 0) {   // both CTAs of the cluster take this branch together
-    if (r == 0 && threadIdx.x < a.H && threadIdx.x < 128) {
-      a.part_ml[(unit * a.H + threadIdx.x) * 2] = -INFINITY;
-      a.part_ml[(unit * a.H + threadIdx.x) * 2 + 1] = 0.f;
+    if (threadIdx.x < a.H && threadIdx.x < 128) {
+      ml[(unit * a.H + threadIdx.x) * 2] = -INFINITY;
+      ml[(unit * a.H + threadIdx.x) * 2 + 1] = 0.f;
     }
     return;
   }
@@ -451,13 +456,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
                             __uint_as_float(o[k + 3]));
         }
       }
-      if (r == 0 && h < a.H) {
-        a.part_ml[(unit * a.H + h) * 2] = m_ref * 0.69314718055994531f;   // natural-log units
-        a.part_ml[(unit * a.H + h) * 2 + 1] = l;
+      if (h < a.H) {
+        ml[(unit * a.H + h) * 2] = m_ref * 0.69314718055994531f;   // natural-log units
+        ml[(unit * a.H + h) * 2 + 1] = l;
       }
-    } else if (r == 0 && h < a.H) {
-      a.part_ml[(unit * a.H + h) * 2] = -INFINITY;
-      a.part_ml[(unit * a.H + h) * 2 + 1] = 0.f;
+    } else if (h < a.H) {
+      ml[(unit * a.H + h) * 2] = -INFINITY;
+      ml[(unit * a.H + h) * 2 + 1] = 0.f;
     }
   }
   tc_fence_before();

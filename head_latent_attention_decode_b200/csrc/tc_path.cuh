@@ -662,6 +662,9 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
   int st;
   // 1. split-KV absorbed attention and the LSE merge -> o_lat (bf16)
   const int R = rkv + dr;
+  const float* sink = h->has_sink ? (const float*)(h->base + h->L.sink) : nullptr;
+  long long ml_r = 0;         // offset of the second CTA's (m, l) copy (head-major kernel)
+  int half_cols = 0;          // latent columns per (m, l) copy (0: one copy)
   const bool latent_ok = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && (((uintptr_t)q_abs) & 15) == 0 &&
                          (((uintptr_t)q_pe) & 15) == 0;
   if (latent_ok && H <= 32) {
@@ -739,6 +742,8 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     ta.rope_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? rkv : 0;
     ta.scale_log2 = h->scale * 1.4426950408889634f;
     ta.part_o = part_o; ta.part_ml = part_ml; ta.flag = flag;
+    ta.ml_r = ml_r = (long long)n * sp * H * 2;
+    half_cols = 256;
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -764,9 +769,8 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     mla_timer_end("attn", s);
     mla_count_launch(1);
   }
-  const float* sink = h->has_sink ? (const float*)(h->base + h->L.sink) : nullptr;
   launch_pdl(attn_combine_kernel<bf16>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits, H,
-             rkv, o_lat, sink);
+             rkv, o_lat, sink, ml_r, half_cols);
   mla_count_launch(1);
   return MLA_OK;
 }
