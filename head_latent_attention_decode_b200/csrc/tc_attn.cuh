@@ -41,9 +41,10 @@ struct TcAttnArgs {
   float* part_o;   // [n, splits, H, 512]
   float* part_ml;  // [n, splits, H, 2], and the same again at part_ml + ml_r
   int* flag;
-  // CTA r of a pair stores its own (m, l) at part_ml + r * ml_r: the two CTAs
-  // add the same two partial scores in a different rounding (own fp32 + peer
-  // f16), so each half of the latent is normalised with its own statistics
+  // head-major kernel: CTA r of the pair stores its own (m, l) at part_ml +
+  // r * ml_r. The two CTAs add the same two partial scores in a different
+  // rounding (own fp32 + peer f16), so each half of the latent is normalised
+  // with its own statistics. (The few-head kernel stores CTA 0's only.)
   long long ml_r;
   // optional tracing: %globaltimer stamps of cluster 0, both CTAs, for the
   // first 64 tiles, [CTA][tile][32]: softmax (head 0) 0 iteration start,
