@@ -41,7 +41,7 @@ sys.path.insert(0, ROOT)
 import head_latent_attention_decode_b200 as mla  # noqa: E402
 from head_latent_attention_decode_b200 import workloads as wl  # noqa: E402
 
-DEFAULT_WORKLOAD = "v2lite_bf16"
+DEFAULT_WORKLOAD = "v3_fp8"
 METRIC_DECODE = "MLA decode tokens/s (one layer step: front-fold + absorbed paged attention + o_proj)"
 METRIC_PREFILL = "MLA prefill TFLOP/s (causal expanded path)"
 METRIC_V4 = "MLA DeepSeek-V4 QKV projection TFLOP/s"

@@ -37,7 +37,7 @@ SYMBOLS = (
     "mla_decode_qkv", "mla_decode_attn", "mla_prefill", "mla_strerror",
     "mla_kernel_launch_count", "mla_set_kernel_timer", "mla_decode_qkv_noalloc",
     "mla_decode_step_host_bytes", "mla_decode_step_host", "mla_rope_cos_sin_inv_freq",
-    "mla_v4_qkv",
+    "mla_v4_qkv", "mla_noalloc_read_device_flag",
 )
 
 MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -106,6 +106,8 @@ def lib() -> ctypes.CDLL:
         L.mla_set_kernel_timer.restype = i
         L.mla_decode_qkv_noalloc.restype = i
         L.mla_decode_qkv_noalloc.argtypes = [vp, vp, i, vp, vp, vp, i, vp, vp, vp, vp]
+        L.mla_noalloc_read_device_flag.restype = i
+        L.mla_noalloc_read_device_flag.argtypes = [ctypes.POINTER(i), vp]
         L.mla_set_kernel_timer.argtypes = [ctypes.c_char_p, vp, vp]
         L.mla_rope_cos_sin_inv_freq.restype = i
         L.mla_rope_cos_sin_inv_freq.argtypes = [vp, i, i, vp, vp, vp, vp]
@@ -224,6 +226,16 @@ def mla_decode_qkv_noalloc(handle, hidden, cos, sin, kv_cache, slot_mapping, q_a
     _check(lib().mla_decode_qkv_noalloc(handle, _ptr(hidden), n, _ptr(cos), _ptr(sin), _ptr(kv_cache),
                                         kv_cache.shape[0], _ptr(slot_mapping), _ptr(q_abs), _ptr(q_pe),
                                         _stream(stream)), "mla_decode_qkv_noalloc")
+
+
+def mla_noalloc_read_device_flag(stream=None) -> int:
+    """Device flag of the last mla_decode_qkv_noalloc call on the current device
+    (synchronises the stream); 0 when that call met no bad slot or timeout."""
+    v = ctypes.c_int(0)
+    st = lib().mla_noalloc_read_device_flag(ctypes.byref(v), _stream(stream))
+    if st not in (MLA_OK, MLA_ERR_DEVICE_FLAG):
+        _check(st, "mla_noalloc_read_device_flag")
+    return v.value
 
 
 def mla_decode_attn(handle, q_abs, q_pe, kv_cache, block_table, context_lens, max_context_len,

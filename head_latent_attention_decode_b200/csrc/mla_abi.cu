@@ -226,6 +226,9 @@ size_t mla_decode_workspace_bytes_internal(const mla_handle* h, int n) {
   return make_ws(h, n, 1).dec_total;
 }
 
+// Commits mla_decode_qkv_noalloc's device array on the current device (mla_noalloc.cu).
+void mla_noalloc_prepare_device();
+
 extern "C" {
 
 const char* mla_strerror(int s) {
@@ -322,6 +325,7 @@ int mla_init_weights(const mla_config* cfg, const mla_weights_desc* w, void* dst
   st = cuda_status();
   if (st == MLA_OK) st = tc_init(h);
   if (st != MLA_OK) { delete h; return st; }
+  mla_noalloc_prepare_device();
   *out = h;
   return MLA_OK;
 }

@@ -28,7 +28,9 @@ static std::mutex g_noalloc_mu;
 static void* g_noalloc_ptr[64] = {nullptr};
 
 // Device address of the scratch on the current device (set up once per
-// device, with that device current).
+// device, with that device current). Looking the symbol up loads the module
+// that holds the array, which is when its device memory is taken: with CUDA's
+// lazy module loading that is the first lookup, not the library's load.
 static int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
@@ -40,6 +42,17 @@ static int noalloc_scratch(void** out) {
   }
   *out = g_noalloc_ptr[dev];
   return MLA_OK;
+}
+
+// Called by mla_init_weights with the handle's device current, so that the
+// array is committed when the first handle on a device is created rather than
+// at the first allocation-free call (a caller whose pool has reserved the rest
+// of the device by then could not take it later). A failure here only defers
+// the lookup to that first call.
+void mla_noalloc_prepare_device() {
+  void* p = nullptr;
+  (void)noalloc_scratch(&p);
+  cudaGetLastError();
 }
 
 extern "C" int mla_decode_qkv_noalloc(mla_handle* h, const void* hidden, int n, const float* cos,
@@ -57,4 +70,16 @@ extern "C" int mla_decode_qkv_noalloc(mla_handle* h, const void* hidden, int n, 
   if (cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
   return mla_decode_qkv(h, hidden, n, cos, sin, kv_cache, n_blocks, slot_mapping, q_abs, q_pe, nullptr, ws,
                         (size_t)MLA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int mla_noalloc_read_device_flag(int* flag_out, void* stream) {
+  if (!flag_out) return MLA_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  const int st = noalloc_scratch(&ws);
+  if (st != MLA_OK) return st;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, (cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
+  *flag_out = v;
+  return v ? MLA_ERR_DEVICE_FLAG : MLA_OK;
 }

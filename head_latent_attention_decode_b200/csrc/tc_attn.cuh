@@ -41,19 +41,10 @@ struct TcAttnArgs {
   float* part_o;   // [n, splits, H, 512]
   float* part_ml;  // [n, splits, H, 2], and the same again at part_ml + ml_r
   int* flag;
-  // head-major kernel: CTA r of the pair stores its own (m, l) at part_ml +
-  // r * ml_r. The two CTAs add the same two partial scores in a different
-  // rounding (own fp32 + peer f16), so each half of the latent is normalised
-  // with its own statistics. (The few-head kernel stores CTA 0's only.)
+  // CTA r of the pair stores its own (m, l) at part_ml + r * ml_r. The two
+  // CTAs add the same two partial scores in a different rounding (own fp32 +
+  // peer f16), so each half of the latent is normalised with its own statistics.
   long long ml_r;
-  // optional tracing: %globaltimer stamps of cluster 0, both CTAs, for the
-  // first 64 tiles, [CTA][tile][32]: softmax (head 0) 0 iteration start,
-  // 2 peer partial arrived, 6 S ready, 7 S read, 11 partials added, 3 peer
-  // buffer freed, 4 P computed, 5 P handed over; sender (the issuing thread)
-  // 12 S ready, 13 S read, 14 peer buffer free, 1 partial sent; MMA thread
-  // 16 S issue starts, 8 S issued, 17 P.V issue starts, 9 P.V issued;
-  // producer 10 tile load issued; [CTA][0][15] unit start. NULL = off.
-  unsigned long long* trace;
 };
 
 constexpr int ATT_NST = 3;                      // tile ring depth
@@ -123,8 +114,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     return;
   }
   const int nkb = (r == 0) ? 5 : 4;
-  unsigned long long* trace = (a.trace && cid == 0) ? a.trace + r * 64 * 32 : nullptr;
-  if (trace && threadIdx.x == 0) trace[15] = global_timer_ns();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ATT_NST; ++i) { mbar_init(full_b + 8 * i, 1); mbar_init(empty_b + 8 * i, 1); }
@@ -173,7 +162,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         // the 4 latent k-blocks of the 64 rows in one box: [8 row octets][4 k-blocks][8 rows][128 B]
         tma_load_4d(dst, &tm_lat, full_b + 8 * st, 0, 0, a.lat_col0 / 64 + 4 * (int)r, (int)(row / 8));
         if (r == 0) tma_load_3d(dst + 4 * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
-        if (trace && t < 64) trace[t * 32 + 10] = global_timer_ns();
       }
       // drain the loads still in flight
       if (r == 0) {
@@ -204,7 +192,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         if (next_s < T && next_s < next_o + 2) {
           const int t = next_s, st = t % ATT_NST, sb = t & 1;
           if (mbar_test(full_b + 8 * st, (t / ATT_NST) & 1) && mbar_test(sp_empty_b + 8 * sb, ((t >> 1) & 1) ^ 1)) {
-            if (trace && t < 64) trace[t * 32 + 16] = global_timer_ns();
             tc_fence_after();
             const uint64_t dt = d_t + (uint64_t)(st * (SM::STAGE / 16));
             const uint32_t d = tmem + ATT_TM_S + 64 * sb;
@@ -220,7 +207,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
               for (int k = 0; k < 4; ++k) mma_bf16(d, d_qr + 2 * k, dr + 2 * k, idesc_s, 1u);
             }
             mma_commit(s_full_b + 8 * sb);
-            if (trace && t < 64) trace[t * 32 + 8] = global_timer_ns();
             ++next_s;
             did = true;
           }
@@ -228,7 +214,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         if (!did && next_o < next_s) {
           const int u = next_o, st = u % ATT_NST, sb = u & 1;
           if (mbar_test(p_full_b + 8 * sb, (u >> 1) & 1)) {
-            if (trace && u < 64) trace[u * 32 + 17] = global_timer_ns();
             tc_fence_after();
             const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
 #pragma unroll
@@ -238,7 +223,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
             mma_commit(o_done);
             mma_commit(sp_empty_b + 8 * sb);
             mma_commit(empty_b + 8 * st);
-            if (trace && u < 64) trace[u * 32 + 9] = global_timer_ns();
             ++next_o;
             did = true;
           }
@@ -271,8 +255,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     for (int k = 0; k < T; ++k) {
       const int kb = k & 1;
       if (!mbar_wait_warp(s_full_b + 8 * kb, (k >> 1) & 1, abort_word, a.flag)) break;
-      const bool trs = trace && issuer && k < 64;
-      if (trs) trace[k * 32 + 12] = global_timer_ns();
       tc_fence_after();
       float v[64];
       const uint32_t sa = tmem + ATT_TM_S + 64 * kb + lane_base;
@@ -281,7 +263,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(s_read_b + 8 * kb);
-      if (trs) trace[k * 32 + 13] = global_timer_ns();
       if (issuer) bulk_wait_read_all();                  // the previous copy has left the staging buffer
       named_bar_sync(2, 128);
       // the partial goes out in f16 (half the distributed-shared-memory bytes of fp32; the
@@ -303,13 +284,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         // the peer has consumed what we sent for tile k - 2 into the same buffer
         const int xb = k & 1;
         bool ok = mbar_wait_cluster(x_free_b + 8 * xb, ((k >> 1) & 1) ^ 1, abort_word, a.flag);
-        if (trs) trace[k * 32 + 14] = global_timer_ns();
         if (ok) {
           bulk_copy_to_peer(peer_x + xb * 16384, stg_s, 16384, peer_x_full + 8 * xb);
           bulk_commit_group();
         }
       }
-      if (trs) trace[k * 32 + 1] = global_timer_ns();
     }
     if (issuer) bulk_wait_read_all();
   } else {
@@ -346,21 +325,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       const int blk = blk_next;
       blk_next = tile_block(t + 1);
       const int valid = (blk >= 0 && blk < a.n_blocks) ? min(64, r1 - (r0 + 64 * t)) : 0;
-      const bool tr = trace && h == 0 && t < 64;
-      if (tr) trace[t * 32 + 0] = global_timer_ns();
       const int xb = t & 1;
       if (h == 0) mbar_arrive_expect_tx(x_full_b + 8 * xb, 16384);
       if (!mbar_wait_warp(x_full_b + 8 * xb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      if (tr) trace[t * 32 + 2] = global_timer_ns();
       if (!mbar_wait_warp(s_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      if (tr) trace[t * 32 + 6] = global_timer_ns();
       tc_fence_after();
       float v[64];
       const uint32_t sp_addr = tmem + ATT_TM_S + 64 * sb + lane_base;
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld16(sp_addr + 16 * c, (uint32_t*)&v[16 * c]);
       tmem_ld_wait();
-      if (tr) trace[t * 32 + 7] = global_timer_ns();
       const uint4* xloc = (const uint4*)(smem + SM::X_OFF + xb * 16384 + h * 128);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -373,10 +347,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
           v[8 * c + 2 * j + 1] += f.y;
         }
       }
-      if (tr) trace[t * 32 + 11] = global_timer_ns();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote_relaxed(peer_x_free + 8 * xb);
-      if (tr) trace[t * 32 + 3] = global_timer_ns();
       // online softmax in log2 units with a lazily moved reference max
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (valid < 64) {
@@ -403,7 +375,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         pk[j >> 1] = *reinterpret_cast<uint32_t*>(&pb);
       }
       const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      if (tr) trace[t * 32 + 4] = global_timer_ns();
       if (__any_sync(0xffffffffu, rescale) && t >= 1) {
         // P.V of the previous tiles must be complete before O is touched
         if (!mbar_wait_warp(o_done, (t - 1) & 1, abort_word, a.flag)) { ok = false; break; }
@@ -438,7 +409,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full_b + 8 * sb);
-      if (tr) trace[t * 32 + 5] = global_timer_ns();
     }
     // every MMA, the last P.V included, has completed once `fin` does (waiting
     // on o_done's parity could pass while an earlier P.V is still running)

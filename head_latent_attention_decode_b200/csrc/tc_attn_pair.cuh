@@ -14,7 +14,8 @@
 //   rows vote whether any score exceeds its head's reference by more than 2^8,
 //   and only then are the column maxima reduced (warp redux and a 4-warp
 //   exchange) and O^T rescaled; per-row partial sums are reduced once at the
-//   end. Both CTAs add the same two partials, so both compute the same P^T
+//   end. Both CTAs add the same two partials, each its own in fp32 and the
+//   peer's in f16, so their P^T agree to the f16 rounding of a partial score
 //   O_r^T += V_r^T . P^T                 2 x (M 128 latent x N NH, K 128 rows),
 //                                        V^T read MN-major from the same tile
 // A CTA keeps 64 KB of a tile until its P.V (half of what one CTA holding the
@@ -88,23 +89,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
   const int r0 = sp * a.chunk, r1 = min(L, r0 + a.chunk);
   const int T = r1 > r0 ? (r1 - r0 + 127) / 128 : 0;
   const long long unit = (long long)b * a.splits + sp;
+  // CTA r stores its own (m, l) at part_ml + r * ml_r: the two CTAs add the
+  // same two partial scores in a different rounding (own fp32 + peer f16), so
+  // their lazily moved reference maxima can differ, and each latent half is
+  // normalised with the statistics of the CTA that accumulated it
+  float* const ml = a.part_ml + r * a.ml_r;
   if (T == 0) {   // both CTAs of the cluster take this branch together
-    if (r == 0 && threadIdx.x < a.H) {
-      a.part_ml[(unit * a.H + threadIdx.x) * 2] = -INFINITY;
-      a.part_ml[(unit * a.H + threadIdx.x) * 2 + 1] = 0.f;
+    if (threadIdx.x < a.H) {
+      ml[(unit * a.H + threadIdx.x) * 2] = -INFINITY;
+      ml[(unit * a.H + threadIdx.x) * 2 + 1] = 0.f;
     }
     return;
   }
-  // optional %globaltimer trace of cluster 0 (its first 64 tiles, [tile][32]):
-  // CTA 0 softmax thread 0: 0 iteration start, 1 early send done, 2 peer
-  // partial in, 3 maxima exchanged, 4 P handed over, 5 late send done; 6 / 7
-  // its S^T(t) ready / peer buffer free when sending; MMA thread: 8 S^T(t)
-  // issued, 9 P.V(t) issued; producer: 11 tile t started, 10 tile t issued;
-  // 12 partials added, 13 column maxima posted, 14 P^T buffer free; per
-  // softmax warp w: 16 + w P handed over, 21 + w peer partial in, 25 + w
-  // maxima exchanged; MMA thread 20 P^T(t) seen; [0][31] kernel start
-  unsigned long long* trace = (a.trace && cid == 0) ? a.trace : nullptr;
-  if (trace && r == 0 && threadIdx.x == 0) trace[31] = global_timer_ns();
   if (threadIdx.x == 0) {
     for (int i = 0; i < NPR; ++i) { mbar_init(full_b + 8 * i, 1); mbar_init(empty_b + 8 * i, 1); }
     mbar_init(rfull, 1);
@@ -150,7 +146,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       int e = 0, ro = 0;
       bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
-        if (trace && r == 0 && t < 64) trace[t * 32 + 11] = global_timer_ns();
         long long row[2];
         for (int hf = 0; hf < 2; ++hf) {
           const int j0 = r0 + 128 * t + 64 * hf;
@@ -176,7 +171,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
           for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(dst + hf * 16384, &tm_lat, fb, 0, 0, a.lat_col0 / 64 + 4 * (int)r + 2 * g, (int)(row[hf] / 8));
         }
-        if (trace && r == 0 && t < 64) trace[t * 32 + 10] = global_timer_ns();
       }
       // let the loads still in flight land before the CTA can exit
       {
@@ -217,7 +211,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
                mbar_wait(full_b + 8 * s1, ((es + 1) / NPR) & 1, abort_word, a.flag) &&
                (!rope || mbar_wait(rfull, ros & 1, abort_word, a.flag));
           if (!ok) break;
-          if (trace && r == 0 && t < 64) trace[t * 32 + 15] = global_timer_ns();
           tc_fence_after();
           const uint32_t d = tm_s + NH * sb;
 #pragma unroll
@@ -237,7 +230,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
             ++ros;
           }
           mma_commit(s_full_b + 8 * sb);
-          if (trace && r == 0 && t < 64) trace[t * 32 + 8] = global_timer_ns();
           es += 2;
         }
         mma_commit(fin_s);
@@ -249,7 +241,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
         for (int u = 0; u < T && ok; ++u) {
           const int sb = u & 1;
           if (!(ok = mbar_wait(p_full_b + 8 * sb, (u >> 1) & 1, abort_word, a.flag))) break;
-          if (trace && r == 0 && u < 64) trace[u * 32 + 20] = global_timer_ns();
           tc_fence_after();
           const uint64_t dp = d_p + (uint64_t)(sb * (2 * QKB / 16));
 #pragma unroll
@@ -260,13 +251,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
             for (int k = 0; k < 8; ++k)
               mma_bf16(tm_o + NH * g, dv + 4096 * k / 16, dp + ((k >> 2) * QKB + 32 * (k & 3)) / 16, idesc_o,
                        (u > 0 || k > 0) ? 1u : 0u);
-            if (g == 0 && trace && r == 0 && u < 64) trace[u * 32 + 29] = global_timer_ns();
             mma_commit(empty_b + 8 * slot);
-            if (g == 0 && trace && r == 0 && u < 64) trace[u * 32 + 30] = global_timer_ns();
           }
           mma_commit(o_done);
           mma_commit(pbuf_free_b + 8 * sb);
-          if (trace && r == 0 && u < 64) trace[u * 32 + 9] = global_timer_ns();
           eo += 2;
         }
         mma_commit(fin);
@@ -282,7 +270,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     const uint32_t peer_x = mapa_shared(x_s, peer), peer_x_full = mapa_shared(x_full_b, peer);
     const uint32_t peer_x_free = mapa_shared(x_free_b, peer);
     const int xsw = (i >> XSH) & (CPR - 1);
-    const bool tr0 = trace && r == 0 && i == 0;
     float m_ref[NH], l_part[NH], cur[NH], nxt[NH];
 #pragma unroll
     for (int h = 0; h < NH; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
@@ -290,7 +277,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     auto fetch_send = [&](int u) -> bool {
       const int sb = u & 1;
       if (!mbar_wait_warp(s_full_b + 8 * sb, (u >> 1) & 1, abort_word, a.flag)) return false;
-      if (tr0 && u < 64) trace[u * 32 + 6] = global_timer_ns();
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < NH / 16; ++c) tmem_ld16(tm_s + NH * sb + lane_base + 16 * c, (uint32_t*)&nxt[16 * c]);
@@ -300,7 +286,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       if (lane == 0) mbar_arrive(s_free_b + 8 * sb);
       // the peer has read what we sent for tile u - 2 out of this buffer
       if (!mbar_wait_cluster_warp(x_free_b + 8 * sb, ((u >> 1) & 1) ^ 1, abort_word, a.flag)) return false;
-      if (tr0 && u < 64) trace[u * 32 + 7] = global_timer_ns();
       // the partial crosses in f16 (half the bytes; partial scores stay far inside its range)
       const uint32_t dst = peer_x + sb * SM::XB + i * (NH * 2);
 #pragma unroll
@@ -328,7 +313,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     int n_slow = 0;   // tiles that needed the column maxima (phases of red2_b)
     for (int t = 0; t < T && ok; ++t) {
       const int sb = t & 1;
-      if (tr0 && t < 64) trace[t * 32 + 0] = global_timer_ns();
       // send the next tile's partial now if its S^T is already there (warp-uniform test)
       if (t + 1 < T && sent == t + 1) {
         const int ready = __shfl_sync(0xffffffffu, lane == 0 ? (int)mbar_test(s_full_b + 8 * ((t + 1) & 1),
@@ -337,7 +321,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
         if (ready) {
           if (!fetch_send(t + 1)) { ok = false; break; }
           sent = t + 2;
-          if (tr0 && t < 64) trace[t * 32 + 1] = global_timer_ns();
         }
       }
       const int valid_rows = min(128, r1 - (r0 + 128 * t));
@@ -346,8 +329,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       // S^T = ours + the peer's partial
       if (i == 0) mbar_arrive_expect_tx(x_full_b + 8 * sb, SM::XB);
       if (!mbar_wait_warp(x_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      if (tr0 && t < 64) trace[t * 32 + 2] = global_timer_ns();
-      if (trace && r == 0 && lane == 0 && t < 64) trace[t * 32 + 21 + warp] = global_timer_ns();
       {
         const uint4* xr = (const uint4*)(smem + SM::X_OFF + sb * SM::XB + i * (NH * 2));
 #pragma unroll
@@ -362,7 +343,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
           }
         }
       }
-      if (tr0 && t < 64) trace[t * 32 + 12] = global_timer_ns();
       // the warp's reads of X have returned (their sums are in registers), so a
       // relaxed arrive suffices; a release at cluster scope would stall the warp
       // until all its earlier memory traffic is visible cluster-wide
@@ -375,13 +355,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
 #pragma unroll
       for (int h = 0; h < NH; ++h) need |= valid && (cur[h] * a.scale_log2 > m_ref[h] + 8.f);
       if (__any_sync(0xffffffffu, need) && lane == 0) vote[sb] = t;
-      if (tr0 && t < 64) trace[t * 32 + 13] = global_timer_ns();
       // rendezvous of the four softmax warps on an mbarrier (a bounded wait, unlike bar.sync)
       __syncwarp();
       if (lane == 0) mbar_arrive(red_b + 8 * sb);
       if (!mbar_wait_warp(red_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      if (tr0 && t < 64) trace[t * 32 + 3] = global_timer_ns();
-      if (trace && r == 0 && lane == 0 && t < 64) trace[t * 32 + 25 + warp] = global_timer_ns();
       float alpha[NH];
       bool rescale = false;
 #pragma unroll
@@ -408,7 +385,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       }
       // P^T(t) into buffer sb once P.V of tile t-2 has released it
       if (!mbar_wait_warp(pbuf_free_b + 8 * sb, ((t >> 1) & 1) ^ 1, abort_word, a.flag)) { ok = false; break; }
-      if (tr0 && t < 64) trace[t * 32 + 14] = global_timer_ns();
       uint8_t* pbuf = smem + SM::P_OFF + sb * 2 * QKB + (i >> 6) * QKB;
       const int col = i & 63;
 #pragma unroll
@@ -449,12 +425,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full_b + 8 * sb);
-      if (tr0 && t < 64) trace[t * 32 + 4] = global_timer_ns();
-      if (trace && r == 0 && lane == 0 && t < 64) trace[t * 32 + 16 + warp] = global_timer_ns();
       if (t + 1 < T && sent == t + 1) {
         if (!fetch_send(t + 1)) { ok = false; break; }
         sent = t + 2;
-        if (tr0 && t < 64) trace[t * 32 + 5] = global_timer_ns();
       }
 #pragma unroll
       for (int h = 0; h < NH; ++h) cur[h] = nxt[h];
@@ -483,17 +456,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
             if (h < a.H) a.part_o[(unit * a.H + h) * 512 + 256 * r + 128 * g + i] = __uint_as_float(o[k]);
           }
         }
-      if (r == 0 && i == 0 && mbar_wait(l_done, 0, abort_word, a.flag)) {
+      if (i == 0 && mbar_wait(l_done, 0, abort_word, a.flag)) {
 #pragma unroll
         for (int h = 0; h < NH; ++h)
           if (h < a.H) {
-            a.part_ml[(unit * a.H + h) * 2] = m_ref[h] * 0.69314718055994531f;
-            a.part_ml[(unit * a.H + h) * 2 + 1] = rl[h] + rl[NH + h] + rl[2 * NH + h] + rl[3 * NH + h];
+            ml[(unit * a.H + h) * 2] = m_ref[h] * 0.69314718055994531f;
+            ml[(unit * a.H + h) * 2 + 1] = rl[h] + rl[NH + h] + rl[2 * NH + h] + rl[3 * NH + h];
           }
       }
-    } else if (r == 0 && i < a.H) {
-      a.part_ml[(unit * a.H + i) * 2] = -INFINITY;
-      a.part_ml[(unit * a.H + i) * 2 + 1] = 0.f;
+    } else if (i < a.H) {
+      ml[(unit * a.H + i) * 2] = -INFINITY;
+      ml[(unit * a.H + i) * 2 + 1] = 0.f;
     }
   }
   tc_fence_before();

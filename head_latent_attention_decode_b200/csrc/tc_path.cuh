@@ -663,7 +663,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
   // 1. split-KV absorbed attention and the LSE merge -> o_lat (bf16)
   const int R = rkv + dr;
   const float* sink = h->has_sink ? (const float*)(h->base + h->L.sink) : nullptr;
-  long long ml_r = 0;         // offset of the second CTA's (m, l) copy (head-major kernel)
+  long long ml_r = 0;         // offset of the second CTA's (m, l) copy (tensor-core kernels)
   int half_cols = 0;          // latent columns per (m, l) copy (0: one copy)
   const bool latent_ok = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && (((uintptr_t)q_abs) & 15) == 0 &&
                          (((uintptr_t)q_pe) & 15) == 0;
@@ -698,6 +698,8 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     ta.rope_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? rkv : 0;
     ta.scale_log2 = h->scale * 1.4426950408889634f;
     ta.part_o = part_o; ta.part_ml = part_ml; ta.flag = flag;
+    ta.ml_r = ml_r = (long long)n * sp * H * 2;   // CTA r's (m, l) copy, one per latent half
+    half_cols = 256;
     static bool attr16[64] = {false}, attr32[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);

@@ -243,17 +243,27 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe,
  * Same computation, arguments and results as mla_decode_qkv (input_norm_w is
  * taken as NULL); the scratch is a static device array of
  * MLA_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
- * process exits. The first call on a device looks up that array's address
- * (cudaGetSymbolAddress) with the device current; make that first call before
- * any stream capture. Returns MLA_ERR_WORKSPACE when the front-fold's
- * workspace for n tokens exceeds the array (for the DeepSeek-V3 shape that
- * allows about 64 tokens per call). All calls share the one array, whose
- * contents persist between calls: each call clears the device flag it holds
- * (so the flag is not readable here), and calls that overlap on the GPU, on
- * any streams, race. Calls no cudaMalloc, cudaFree or allocating routine. */
+ * process exits. The array's device memory is taken when the library first
+ * looks up its address (cudaGetSymbolAddress) on a device, with that device
+ * current: mla_init_weights does so for its device, so the memory is committed
+ * when the first handle is created; if that lookup failed, the first call
+ * here repeats it, so make that first call before any stream capture.
+ * Returns MLA_ERR_WORKSPACE when the front-fold's workspace for n tokens
+ * exceeds the array (for the DeepSeek-V3 shape that allows about 64 tokens
+ * per call). All calls share the one array, whose contents persist between
+ * calls: each call clears the device flag it holds before its kernels run
+ * (read it with mla_noalloc_read_device_flag), and calls that overlap on the
+ * GPU, on any streams, race. Calls no cudaMalloc, cudaFree or allocating
+ * routine. */
 int mla_decode_qkv_noalloc(mla_handle* h, const void* hidden, int n, const float* cos,
                            const float* sin, void* kv_cache, int n_blocks,
                            const int32_t* slot_mapping, void* q_abs, void* q_pe, void* stream);
+
+/* The device flag of the last mla_decode_qkv_noalloc call on the current
+ * device (bad slot: that row was not written; wait timeout: q_abs / q_pe are
+ * incomplete), copied to *flag_out after synchronising `stream`. Returns
+ * MLA_ERR_DEVICE_FLAG when it is non-zero, MLA_OK otherwise. */
+int mla_noalloc_read_device_flag(int* flag_out, void* stream);
 
 /* ---- one decode step from host memory ------------------------------------------ */
 

@@ -397,6 +397,39 @@ def test_scatter_writes_only_mapped_rows():
     np.testing.assert_array_equal(flat_new[untouched], flat_old[untouched])
 
 
+@pytest.mark.parametrize("shape", [SMALL, SMALL_NOQ])
+@pytest.mark.parametrize("layout", [ref.LATENT_FIRST, ref.PE_FIRST])
+def test_fill_cache_by_projection_matches_brute_force(shape, layout):
+    """The earlier rows of each sequence (positions 0..L-2, the hidden state of
+    position p projected, normed, rotated at p and written at its slot) against
+    the literal loops, which take one token per position through the same
+    front-fold and scatter; every other row keeps its value."""
+    w = wl.Workload("t", shape, "decode", batch=3, ctx_lo=2, ctx_hi=7, cache_fill="project", seed=11)
+    inp = wl.make_decode_inputs(w)
+    W = _weights(shape, 11)
+    got = ref.fill_cache_by_projection(shape, W, inp.cache, inp.fill_hidden, inp.fill_slots, layout)
+    rows = inp.cache.reshape(-1, shape.kv_row_dim).tolist()
+    shifted = [list(r) for r in rows]
+    for xs, slots in zip(inp.fill_hidden, inp.fill_slots):
+        m = len(slots)
+        if m == 0:
+            continue
+        for pos0, dst in ((0, rows), (1, shifted)):   # pos0 = 1: the off-by-one reading
+            _, _, _, _, new = brute.decode_step(shape, W, xs, np.arange(pos0, pos0 + m), dst,
+                                                [[0]] * m, [1] * m, slots, layout)
+            dst[:] = new
+    got_flat = got.reshape(-1, shape.kv_row_dim)
+    np.testing.assert_allclose(got_flat, np.array(rows), rtol=0, atol=1e-12)
+    written = {int(s) for sl in inp.fill_slots for s in sl}
+    assert written and len(written) == sum(len(s) for s in inp.fill_slots)
+    old = inp.cache.reshape(-1, shape.kv_row_dim)
+    for i in range(len(old)):
+        if i not in written:
+            np.testing.assert_array_equal(got_flat[i], old[i])
+    # positions shifted by one would move every rotated k_pe: the pin sees it
+    assert np.max(np.abs(got_flat - np.array(shifted))) > 1e-3
+
+
 def test_cache_row_layouts():
     c, kpe = np.array([1.0, 2, 3]), np.array([8.0, 9])
     np.testing.assert_array_equal(ref.cache_row(c, kpe, ref.LATENT_FIRST), [1, 2, 3, 8, 9])
