@@ -107,7 +107,7 @@ static WeightLayout make_layout(const mla_config* c) {
 // [0, 256): device flag (int32 at 0) and counters. Then decode and prefill
 // scratch share one region (calls on one workspace are stream-ordered).
 struct WsLayout {
-  size_t Y1, qn, Q, part_o, part_ml, o_lat, head, xn;         // decode
+  size_t Y1, qn, Q, part_o, part_ml, nseg, o_lat, head, xn;   // decode
   size_t pY1, pqn, pQ, pcn, pkpe, pKV, phead, pDQ;             // prefill
   size_t tc;                                                   // tensor-core path scratch
   size_t dec_total;                                            // what the decode calls need
@@ -117,7 +117,7 @@ struct WsLayout {
 
 static int decode_splits(int max_ctx) {
   const int c = (int)cdiv(max_ctx, 256);
-  return c < 1 ? 1 : (c > 16 ? 16 : c);
+  return c < 2 ? 2 : (c > 16 ? 16 : c);
 }
 
 static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
@@ -134,6 +134,7 @@ static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
   W.Q = put((size_t)n * L.Hq * 4);
   W.part_o = put((size_t)n * W.splits * H * rkv * 4);
   W.part_ml = put((size_t)n * W.splits * H * 2 * 4 * 2);   // one (m, l) copy per CTA of a pair
+  W.nseg = put((size_t)n * 4);                                // split partials per sequence
   W.o_lat = put((size_t)n * H * rkv * a);
   W.head = put((size_t)n * H * dv * a);
   W.xn = put((size_t)n * c->hidden * a);
@@ -471,7 +472,7 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
     const int r = tc_decode_attn(h, q_abs, q_pe, kv_cache, n_blocks, block_table, max_blocks_per_seq,
                                  context_lens, max_context_len, n, out, head, wsb, W.tc, s,
                                  (float*)(wsb + W.part_o), (float*)(wsb + W.part_ml), W.splits,
-                                 (bf16*)(wsb + W.o_lat));
+                                 (bf16*)(wsb + W.o_lat), (int*)(wsb + W.nseg));
     return r != MLA_OK ? r : cuda_status();
   }
   void* o_lat = wsb + W.o_lat;
@@ -479,7 +480,8 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
     // tensor-core attention (bf16 activations) ahead of CUDA-core W_UV / o_proj
     const int r = tc_attention_core(h, q_abs, q_pe, kv_cache, n_blocks, block_table, max_blocks_per_seq,
                                     context_lens, max_context_len, n, (float*)(wsb + W.part_o),
-                                    (float*)(wsb + W.part_ml), W.splits, (bf16*)o_lat, flag, s);
+                                    (float*)(wsb + W.part_ml), W.splits, (bf16*)o_lat, flag,
+                                    (int*)(wsb + W.nseg), s);
     if (r != MLA_OK) return r;
   } else {
     AttnArgs p{};
@@ -499,8 +501,8 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
     count_launch();
     dim3 cg(n, H);
     const float* sink = h->has_sink ? (const float*)(h->base + L.sink) : nullptr;
-    if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat, sink, 0, 0);
-    else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat, sink, 0, 0);
+    if (ta == 0) attn_combine_kernel<float><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (float*)o_lat, sink, 0, 0, nullptr);
+    else attn_combine_kernel<bf16><<<cg, 128, 0, s>>>(p.part_o, p.part_ml, W.splits, H, rkv, (bf16*)o_lat, sink, 0, 0, nullptr);
     count_launch();
   }
   // head_out[h] = o_lat[h] @ W_UV[h]

@@ -405,22 +405,25 @@ __global__ void __launch_bounds__(256) attn_decode_simt_kernel(AttnArgs p) {
 // denominator gains e^{z_h - M}. Kernels that split the latent columns over a
 // CTA pair store one (m, l) copy per CTA: columns c >= half_cols then use the
 // copy ml_r floats further on (half_cols = 0: one copy for all columns).
+// nseg (optional): sequence t has nseg[t] partials, in its first split slots;
+// otherwise all n_splits slots are read and empty ones carry l = 0.
 // grid (n, H), 128 threads x 4 consecutive columns (r_kv <= 512, r_kv % 4 == 0).
 // Writes o_lat [n, H, r_kv] in act dtype.
 template <typename T>
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, const float* part_ml, int n_splits,
                                                            int H, int r_kv, T* o_lat, const float* sink,
-                                                           long long ml_r, int half_cols) {
+                                                           long long ml_r, int half_cols, const int* nseg) {
   griddep_wait();
   griddep_launch_dependents();
   __shared__ float wsh[2][64];
   __shared__ float inv_sh[2];
   const int t = blockIdx.x, h = blockIdx.y;
+  const int used = nseg ? min(nseg[t], n_splits) : n_splits;   // slots holding this sequence's partials
   const int warp = threadIdx.x >> 5;
   if (warp < (half_cols > 0 ? 2 : 1)) {   // warp w: the weights of stats copy w
     const float* ml = part_ml + warp * ml_r;
     float M = -INFINITY;
-    for (int s = threadIdx.x & 31; s < n_splits; s += 32) {
+    for (int s = threadIdx.x & 31; s < used; s += 32) {
       const long long base = ((long long)t * n_splits + s) * H + h;
       if (ml[base * 2 + 1] > 0.f) M = fmaxf(M, ml[base * 2]);
     }
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, 
     const float z = sink ? sink[h] : -INFINITY;
     M = fmaxf(M, z);
     float den = ((threadIdx.x & 31) == 0 && z > -INFINITY) ? __expf(z - M) : 0.f;
-    for (int s = threadIdx.x & 31; s < n_splits; s += 32) {
+    for (int s = threadIdx.x & 31; s < used; s += 32) {
       const long long base = ((long long)t * n_splits + s) * H + h;
       const float l = ml[base * 2 + 1];
       const float w = (l > 0.f) ? __expf(ml[base * 2] - M) : 0.f;
@@ -443,7 +446,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* part_o, 
   if (c >= r_kv) return;
   const int cp = (half_cols > 0 && c >= half_cols) ? 1 : 0;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int ns = n_splits < 64 ? n_splits : 64;
+  const int ns = used < 64 ? used : 64;
 #pragma unroll 4
   for (int s = 0; s < ns; ++s) {
     const float w = wsh[cp][s];

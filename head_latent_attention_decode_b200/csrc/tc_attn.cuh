@@ -2,27 +2,35 @@
 // qk_rope 64 (the DeepSeek MLA latent), bf16 cache with blocks of a multiple
 // of 64 rows.
 //
-// One 2-CTA cluster per (sequence, KV split). All heads of the token form the
-// MMA's M = 128 rows (fewer heads are padded with zeros). CTA r owns latent
-// columns [256 r, 256 r + 256); CTA 0 also owns the 64 rotary columns. Per
-// 64-row cache tile:
-//   S_r = [q_abs | q_pe]_r . tile_r^T      (tcgen05, M 128 x N 64, K 256 / 320;
-//                                          the latent part of Q lives in TMEM)
-//   S   = S_0 + S_1                        (the partials swap through DSMEM in f16,
-//                                          into two alternating buffers)
-//   online softmax, one thread per head (nothing to reduce across threads),
-//   lazy rescale of the TMEM accumulator when the max grows by more than 2^8;
-//   P (bf16) is written back into TMEM over S
-//   O_r += P . V_r                         (tcgen05 with A = P in TMEM, M 128 x
-//                                          N 256, K 64; V = the same shared-memory
-//                                          tile read MN-major)
-// Every cache byte is read from HBM once, O (128 x 512 fp32) is split over the
-// two CTAs' TMEM, and a 3-deep ring of tiles keeps loads in flight while the
-// MMA thread issues S of later tiles ahead of P.V of earlier ones. Warps 0-3
-// run the softmax, warps 6-9 send each tile's partial scores to the peer as
-// soon as S lands, warp 4 issues TMA and warp 5 the MMAs. Partials
-// (unnormalised O, reference max, sum) go to the workspace and
-// attn_combine_kernel merges the splits.
+// Persistent and balanced: the batch's 64-row cache tiles, sequence after
+// sequence, form one list, and 2-CTA cluster c takes the c-th equal slice of
+// it (so every SM pair streams the same number of tiles whatever the context
+// lengths). The part of a sequence inside one slice is a segment; each
+// segment leaves one split partial (unnormalised O, reference max, sum), and
+// attn_combine_kernel merges a sequence's segments.
+//
+// Per tile: all heads of the token form the MMA's M = 128 rows (fewer heads
+// are padded with zeros). CTA r owns latent columns [256 r, 256 r + 256) of
+// every tile and the 64 rotary columns of the tiles with odd-even index r:
+//   S_r = [q_abs | q_pe]_r . tile_r^T      (tcgen05, M 128 x N 64, K 256 or 320;
+//                                          Q lives in TMEM)
+//   S   = S_r + S_peer                     (the partials swap through DSMEM in
+//                                          f16, into two alternating buffers)
+//   online softmax, two threads per head (each half of the tile's 64 columns;
+//   the halves' maxima meet in shared memory), with a lazily moved reference
+//   max: the accumulator is rescaled only when a head's max grows by more than
+//   2^8; P (bf16) is written over the peer partial it was computed from, in
+//   the MMA's operand layout
+//   O_r += P . V_r                         (tcgen05, A = P from shared memory,
+//                                          M 128 x N 256, K 64; V = the same
+//                                          shared-memory tile read MN-major)
+// Every cache byte is read from HBM once and O (128 x 512 fp32) is split over
+// the two CTAs' TMEM. A tile's ring stage is held from its load until its
+// P.V, so the shared memory left over by the exchange buffers goes to a
+// 4-deep ring; the S buffer is released as soon as the softmax and the sender
+// have read it. Warps 0-7 run the softmax (warp w: TMEM lane quarter w % 4,
+// column half w / 4), warp 8 issues TMA, warp 9 the MMAs, and warps 10-13 send
+// each tile's partial scores to the peer as soon as S lands.
 #pragma once
 
 #include "tc_common.cuh"
@@ -45,92 +53,152 @@ struct TcAttnArgs {
   // CTAs add the same two partial scores in a different rounding (own fp32 +
   // peer f16), so each half of the latent is normalised with its own statistics.
   long long ml_r;
+  // balanced schedule (head-major kernel): `units` clusters, each a slice of at
+  // least `min_per` tiles (which keeps every sequence within `splits` segments);
+  // nseg[b] receives the number of segments (split partials) of sequence b
+  const bf16* q_pe;   // [n, H, 64]
+  int units, min_per;
+  int* nseg;
 };
 
-constexpr int ATT_NST = 3;                      // tile ring depth
-constexpr int ATT_THREADS = 320;                // 4 softmax, 1 TMA, 1 MMA, 4 sender warps
+constexpr int ATT_NST = 4;                      // tile ring depth
+constexpr int ATT_THREADS = 448;                // 8 softmax, 1 TMA, 1 MMA, 4 sender warps
+constexpr int ATT_MAX_SEQ = 256;                // sequences per call (the prefix table in shared memory)
 struct AttnSmem {
   static constexpr int STAGE = 5 * 8192;        // 4 latent + 1 rope slot of [64 rows x 64 cols] bf16
   static constexpr int TILE_OFF = 0;
-  static constexpr int QR_OFF = ATT_NST * STAGE;  // q_pe [128 x 64] bf16 (CTA 0)
-  static constexpr int X_OFF = QR_OFF + 16384;    // 2 x [128 x 64] f16, the peer's partial S (double-buffered)
+  static constexpr int X_OFF = ATT_NST * STAGE;   // 2 x [128 x 64] f16 peer partial S, then P (bf16) over it
   static constexpr int STG_OFF = X_OFF + 32768;   // [128 x 64] f16, our partial on its way out
-  static constexpr int BAR_OFF = STG_OFF + 16384;
-  static constexpr int SIZE = 1024 + BAR_OFF + 256;
+  static constexpr int RED_OFF = STG_OFF + 16384; // [2 tiles][2 halves][128] fp32 half-row maxima, then [128] l
+  static constexpr int PREF_OFF = RED_OFF + 2 * 2 * 128 * 4 + 128 * 4;   // [ATT_MAX_SEQ + 1] tile prefix sums
+  static constexpr int BAR_OFF = PREF_OFF + (ATT_MAX_SEQ + 4) * 4;
+  static constexpr int SIZE = 1024 + BAR_OFF + 512;
 };
-// TMEM columns: Q latent [0,128) (bf16 pairs), S/P buffers [128,192) [192,256), O [256,512)
-constexpr uint32_t ATT_TM_Q = 0, ATT_TM_S = 128, ATT_TM_O = 256;
+// TMEM columns: Q latent [0,128) and q_pe [128,160) (bf16 pairs), S [192,256), O [256,512)
+constexpr uint32_t ATT_TM_Q = 0, ATT_TM_QPE = 128, ATT_TM_S = 192, ATT_TM_O = 256;
 
-__device__ __forceinline__ int attn_tile_rows(const TcAttnArgs& a, int b, int j0, int r1, long long* row) {
-  const int blk = a.block_table[(long long)b * a.mbps + j0 / a.bs];
-  if (blk < 0 || blk >= a.n_blocks) {
-    *row = -64;
-    return -1;
+// Walks a cluster's slice of the batch's tile list: sequence b, its tile lt.
+struct TileWalk {
+  const int* pref;   // pref[b] = tiles of sequences 0..b-1 (shared memory)
+  int n, b, lt;
+  __device__ void start(int g) {
+    b = 0;
+    while (b < n && pref[b + 1] <= g) ++b;
+    lt = g - pref[b];
   }
-  *row = (long long)blk * a.bs + (j0 % a.bs);
-  return min(64, r1 - j0);
+  __device__ bool seg_last() const { return pref[b] + lt + 1 == pref[b + 1]; }
+  __device__ void next() {
+    if (seg_last()) {
+      ++b;
+      while (b < n && pref[b + 1] == pref[b]) ++b;
+      lt = 0;
+    } else {
+      ++lt;
+    }
+  }
+};
+
+// Context length of sequence b as the schedule counts it (0 when invalid).
+__device__ __forceinline__ int attn_seq_len(const TcAttnArgs& a, int b) {
+  const int L = a.ctx[b];
+  return (L < 1 || L > a.max_ctx || L > a.mbps * a.bs) ? 0 : L;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
-    tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_qpe, const __grid_constant__ CUtensorMap tm_cache,
-                          const __grid_constant__ CUtensorMap tm_lat, TcAttnArgs a) {
+    tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_lat,
+                          TcAttnArgs a) {
   using SM = AttnSmem;
   griddep_wait();   // the inputs all come from the stream's earlier kernels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t tile_s = sbase + SM::TILE_OFF, qr_s = sbase + SM::QR_OFF, x_s = sbase + SM::X_OFF;
+  const uint32_t tile_s = sbase + SM::TILE_OFF, x_s = sbase + SM::X_OFF;
+  float* red = (float*)(smem + SM::RED_OFF);      // [tile & 1][half][head]
+  float* red_l = red + 2 * 2 * 128;                // [head]: the second half's row sum
+  int* pref = (int*)(smem + SM::PREF_OFF);
   const uint32_t bar = sbase + SM::BAR_OFF;
   // barriers (8 B each)
-  const uint32_t full_b = bar;                 // [ATT_NST] tile landed
-  const uint32_t empty_b = bar + 8 * ATT_NST;  // [ATT_NST] tile consumed by P.V
-  const uint32_t s_full_b = bar + 16 * ATT_NST;        // [2]
-  const uint32_t p_full_b = s_full_b + 16;             // [2]
-  const uint32_t sp_empty_b = p_full_b + 16;           // [2] S/P buffer free (P.V done)
-  const uint32_t q_ready = sp_empty_b + 16, qr_full = q_ready + 8, o_done = qr_full + 8;
-  const uint32_t x_full_b = o_done + 8, x_free_b = x_full_b + 16, fin = x_free_b + 16;   // x_full[2], x_free[2]
-  const uint32_t s_read_b = fin + 8;   // [2] the sender has read S(t) out of TMEM
-  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 192);
-  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 196);
+  const uint32_t full_b = bar;                        // [ATT_NST] tile landed
+  const uint32_t empty_b = bar + 8 * ATT_NST;         // [ATT_NST] tile consumed by P.V
+  const uint32_t s_full = bar + 16 * ATT_NST;         // S_r(i) complete
+  const uint32_t s_free = s_full + 8;                 // S read by the 8 softmax and 4 sender warps
+  const uint32_t p_full_b = s_free + 8;               // [2] P(i) in shared memory (8 softmax warps)
+  const uint32_t x_full_b = p_full_b + 16;            // [2] peer partial landed
+  const uint32_t x_free_b = x_full_b + 16;            // [2] the peer's P.V has released its buffer
+  const uint32_t q_ready = x_free_b + 16;             // Q of the next segment in TMEM (8 softmax warps)
+  const uint32_t o_done = q_ready + 8;                // each P.V
+  const uint32_t o_seg = o_done + 8;                  // the last P.V of a segment
+  const uint32_t o_free = o_seg + 8;                  // O of a segment read out (8 softmax warps)
+  const uint32_t fin = o_free + 8;
+  const uint32_t xch_b = fin + 8;                     // [4 quarters][2] the two halves' maxima posted
+  const uint32_t l_done = xch_b + 64;                 // [4] the second half's row sums posted
+  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 320);
+  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 324);
 
   const uint32_t r = cluster_ctarank(), peer = r ^ 1u;
-  const int cid = blockIdx.x >> 1;
-  const int b = cid / a.splits, sp = cid % a.splits;
+  const int c = blockIdx.x >> 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int L = a.ctx[b];
-  if (L < 1 || L > a.max_ctx || L > a.mbps * a.bs) {
-    if (threadIdx.x == 0 && r == 0 && sp == 0) set_flag(a.flag, MLA_FLAG_BAD_CONTEXT);
-    L = 0;
-  }
-  const int r0 = sp * a.chunk, r1 = min(L, r0 + a.chunk);
-  const int T = r1 > r0 ? (r1 - r0 + 63) / 64 : 0;
-  const long long unit = (long long)b * a.splits + sp;
-  float* const ml = a.part_ml + r * a.ml_r;   // this CTA's (m, l) copy
-  if (T == 0) {   // both CTAs of the cluster take this branch together
-    if (threadIdx.x < a.H && threadIdx.x < 128) {
-      ml[(unit * a.H + threadIdx.x) * 2] = -INFINITY;
-      ml[(unit * a.H + threadIdx.x) * 2 + 1] = 0.f;
+
+  // ---- the schedule: tile prefix over the batch, then this cluster's slice ----
+  if (warp == 0) {
+    int cnt[8], sum = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int b = 8 * lane + k;
+      int T = 0;
+      if (b < a.n) {
+        const int L = attn_seq_len(a, b);
+        if (L == 0 && c == 0 && r == 0) set_flag(a.flag, MLA_FLAG_BAD_CONTEXT);
+        T = (L + 63) / 64;
+      }
+      cnt[k] = T;
+      sum += T;
     }
-    return;
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int b = 8 * lane + k;
+      if (b < a.n) pref[b] = run;
+      run += cnt[k];
+    }
+    if (lane == 31) pref[a.n] = incl;   // the batch's tile count
   }
-  const int nkb = (r == 0) ? 5 : 4;
+  __syncthreads();
+  const int total = pref[a.n];
+  int per = (total + a.units - 1) / a.units;
+  if (per < a.min_per) per = a.min_per;
+  const int g0 = c * per, g1 = min(total, g0 + per);
+  if (blockIdx.x == 0) {   // segments of each sequence, for the merge
+    for (int b = threadIdx.x; b < a.n; b += blockDim.x) {
+      const int T = pref[b + 1] - pref[b];
+      a.nseg[b] = T > 0 ? (pref[b] + T - 1) / per - pref[b] / per + 1 : 0;
+    }
+  }
+  if (g0 >= g1) return;   // both CTAs of the cluster take this branch together
+  const int N = g1 - g0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ATT_NST; ++i) { mbar_init(full_b + 8 * i, 1); mbar_init(empty_b + 8 * i, 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 12);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full_b + 8 * i, 1);
-      mbar_init(p_full_b + 8 * i, 128);
-      mbar_init(sp_empty_b + 8 * i, 1);
-    }
-    mbar_init(q_ready, 128);
-    mbar_init(qr_full, 1);
-    mbar_init(o_done, 1);
-    for (int i = 0; i < 2; ++i) {
+      mbar_init(p_full_b + 8 * i, 8);
       mbar_init(x_full_b + 8 * i, 1);
-      mbar_init(x_free_b + 8 * i, 4);
+      mbar_init(x_free_b + 8 * i, 1);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(s_read_b + 8 * i, 128);
+    mbar_init(q_ready, 8);
+    mbar_init(o_done, 1);
+    mbar_init(o_seg, 1);
+    mbar_init(o_free, 8);
     mbar_init(fin, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(xch_b + 8 * i, 2);
+    for (int i = 0; i < 4; ++i) mbar_init(l_done + 8 * i, 1);
     *abort_word = 0;
     fence_mbar_init();
   }
@@ -142,88 +210,94 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       prefetch_tmap(&tm_cache);
       prefetch_tmap(&tm_lat);
-      if (r == 0) {
-        mbar_arrive_expect_tx(qr_full, 16384);
-        tma_load_3d(qr_s, &tm_qpe, qr_full, 0, b * a.H, 0);
-      }
-      int t = 0;
-      for (; t < T; ++t) {
-        const int st = t % ATT_NST;
-        if (!mbar_wait(empty_b + 8 * st, ((t / ATT_NST) & 1) ^ 1, abort_word, a.flag)) break;
-        long long row;
-        if (attn_tile_rows(a, b, r0 + 64 * t, r1, &row) < 0 && r == 0) set_flag(a.flag, MLA_FLAG_BAD_BLOCK);
-        mbar_arrive_expect_tx(full_b + 8 * st, nkb * 8192);
+      TileWalk w{pref, a.n, 0, 0};
+      w.start(g0);
+      int i = 0;
+      for (; i < N; ++i, w.next()) {
+        const int st = i % ATT_NST;
+        if (!mbar_wait(empty_b + 8 * st, ((i / ATT_NST) & 1) ^ 1, abort_word, a.flag)) break;
+        const int j0 = 64 * w.lt;
+        const int blk = a.block_table[(long long)w.b * a.mbps + j0 / a.bs];
+        long long row = -64;
+        if (blk >= 0 && blk < a.n_blocks) row = (long long)blk * a.bs + (j0 % a.bs);
+        else if (r == 0) set_flag(a.flag, MLA_FLAG_BAD_BLOCK);
+        const bool rope = (i & 1) == (int)r;
+        mbar_arrive_expect_tx(full_b + 8 * st, rope ? 5 * 8192 : 4 * 8192);
         const uint32_t dst = tile_s + st * SM::STAGE;
         // the 4 latent k-blocks of the 64 rows in one box: [8 row octets][4 k-blocks][8 rows][128 B]
         tma_load_4d(dst, &tm_lat, full_b + 8 * st, 0, 0, a.lat_col0 / 64 + 4 * (int)r, (int)(row / 8));
-        if (r == 0) tma_load_3d(dst + 4 * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
+        if (rope) tma_load_3d(dst + 4 * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
       }
       // drain the loads still in flight
-      if (r == 0) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(qr_full, 0)) if (global_timer_ns() - t0 > WAIT_LIMIT_NS) break;
-      }
-      for (int u = (t > ATT_NST ? t - ATT_NST : 0); u < t; ++u) {
+      for (int u = (i > ATT_NST ? i - ATT_NST : 0); u < i; ++u) {
         const uint64_t t1 = global_timer_ns();
         while (!mbar_try_wait(full_b + 8 * (u % ATT_NST), (u / ATT_NST) & 1))
           if (global_timer_ns() - t1 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
       }
     }
-  } else if (warp == 5) {
-    // ---------------- MMA issuer: S runs up to two tiles ahead of P.V ----------------
+  } else if (warp == 9) {
+    // ---------------- MMA issuer: P.V of the oldest tile first, else the next S ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64);
       constexpr uint32_t idesc_o = idesc_bf16(128, 256, 1);
-      bool ok = mbar_wait(q_ready, 0, abort_word, a.flag);
-      if (ok && r == 0) ok = mbar_wait(qr_full, 0, abort_word, a.flag);
-      tc_fence_after();
       // descriptors built once; stages and k-steps add their byte offset >> 4
       const uint64_t d_t = sdesc_sw128_sbo(tile_s, 4096), d_rope = sdesc_sw128(tile_s + 4 * 8192);
-      const uint64_t d_qr = sdesc_sw128(qr_s), d_v = sdesc_sw128_mn_sbo(tile_s, 1024, 4096);
-      int next_s = 0, next_o = 0;
+      const uint64_t d_v = sdesc_sw128_mn_sbo(tile_s, 1024, 4096), d_p = sdesc_sw128(x_s);
+      TileWalk ws{pref, a.n, 0, 0}, wo{pref, a.n, 0, 0};
+      ws.start(g0);
+      wo.start(g0);
+      int next_s = 0, next_o = 0, ks = 0, ko = 0;
+      bool ok = true;
       uint64_t t_last = global_timer_ns();
-      while (ok && next_o < T) {
+      while (ok && next_o < N) {
         bool did = false;
-        if (next_s < T && next_s < next_o + 2) {
-          const int t = next_s, st = t % ATT_NST, sb = t & 1;
-          if (mbar_test(full_b + 8 * st, (t / ATT_NST) & 1) && mbar_test(sp_empty_b + 8 * sb, ((t >> 1) & 1) ^ 1)) {
+        if (next_o < next_s) {
+          const int u = next_o, st = u % ATT_NST, xb = u & 1;
+          const bool first = (u == 0 || wo.lt == 0), last = (u == N - 1 || wo.seg_last());
+          if (mbar_test(p_full_b + 8 * xb, (u >> 1) & 1) && (!first || ko == 0 || mbar_test(o_free, (ko - 1) & 1))) {
+            tc_fence_after();
+            const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
+            const uint64_t dp = d_p + (uint64_t)(xb * (16384 / 16));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_bf16(tmem + ATT_TM_O, dp + 2 * k, dv + 8192 * k / 16, idesc_o, (!first || k > 0) ? 1u : 0u);
+            mma_commit(o_done);
+            mma_commit(empty_b + 8 * st);
+            mma_commit_cta_mask(x_free_b + 8 * xb, (uint16_t)(1u << peer));   // our buffer xb is the peer's to fill
+            if (last) { mma_commit(o_seg); ++ko; }
+            wo.next();
+            ++next_o;
+            did = true;
+          }
+        }
+        if (next_s < N) {
+          const int t = next_s, st = t % ATT_NST;
+          const bool first = (t == 0 || ws.lt == 0), last = (t == N - 1 || ws.seg_last());
+          if (mbar_test(full_b + 8 * st, (t / ATT_NST) & 1) && mbar_test(s_free, (t & 1) ^ 1) &&
+              (!first || mbar_test(q_ready, ks & 1))) {
             tc_fence_after();
             const uint64_t dt = d_t + (uint64_t)(st * (SM::STAGE / 16));
-            const uint32_t d = tmem + ATT_TM_S + 64 * sb;
+            const uint32_t d = tmem + ATT_TM_S;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 mma_bf16_ts(d, tmem + ATT_TM_Q + 32 * j + 8 * k, dt + (j * 1024 + 32 * k) / 16, idesc_s,
                             (j > 0 || k > 0) ? 1u : 0u);
-            if (r == 0) {
+            if ((t & 1) == (int)r) {
               const uint64_t dr = d_rope + (uint64_t)(st * (SM::STAGE / 16));
 #pragma unroll
-              for (int k = 0; k < 4; ++k) mma_bf16(d, d_qr + 2 * k, dr + 2 * k, idesc_s, 1u);
+              for (int k = 0; k < 4; ++k) mma_bf16_ts(d, tmem + ATT_TM_QPE + 8 * k, dr + 2 * k, idesc_s, 1u);
             }
-            mma_commit(s_full_b + 8 * sb);
+            mma_commit(s_full);
+            if (last) ++ks;
+            ws.next();
             ++next_s;
-            did = true;
-          }
-        }
-        if (!did && next_o < next_s) {
-          const int u = next_o, st = u % ATT_NST, sb = u & 1;
-          if (mbar_test(p_full_b + 8 * sb, (u >> 1) & 1)) {
-            tc_fence_after();
-            const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_bf16_ts(tmem + ATT_TM_O, tmem + ATT_TM_S + 64 * sb + 8 * k, dv + 8192 * k / 16, idesc_o,
-                          (u > 0 || k > 0) ? 1u : 0u);
-            mma_commit(o_done);
-            mma_commit(sp_empty_b + 8 * sb);
-            mma_commit(empty_b + 8 * st);
-            ++next_o;
             did = true;
           }
         }
@@ -236,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
           set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT);
           ok = false;
         } else {
-          __nanosleep(32);   // leave the issue slots to the softmax warp on this sub-partition
+          __nanosleep(32);   // leave the issue slots to the softmax warps on this sub-partition
         }
       }
       mma_commit(fin);
@@ -244,47 +318,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       while (!mbar_try_wait(fin, 0))
         if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
     }
-  } else if (warp >= 6) {
-    // ---------------- senders: S_r(k) -> staging -> one bulk copy into the peer's X ----------------
+  } else if (warp >= 10) {
+    // ---------------- senders: S_r(i) -> staging -> one bulk copy into the peer's X ----------------
     const int h = 32 * (warp & 3) + lane;                 // TMEM lane quarter of this warp
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const bool issuer = (warp == 6 && lane == 0);
+    const bool issuer = (warp == 10 && lane == 0);
     const uint32_t peer_x = mapa_shared(x_s, peer), peer_x_full = mapa_shared(x_full_b, peer);
     const uint32_t stg_s = sbase + SM::STG_OFF;
     uint4* stg_row = (uint4*)(smem + SM::STG_OFF + h * 128);
-    for (int k = 0; k < T; ++k) {
-      const int kb = k & 1;
-      if (!mbar_wait_warp(s_full_b + 8 * kb, (k >> 1) & 1, abort_word, a.flag)) break;
+    for (int i = 0; i < N; ++i) {
+      if (!mbar_wait_warp(s_full, i & 1, abort_word, a.flag)) break;
       tc_fence_after();
       float v[64];
-      const uint32_t sa = tmem + ATT_TM_S + 64 * kb + lane_base;
+      const uint32_t sa = tmem + ATT_TM_S + lane_base;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(sa + 16 * c, (uint32_t*)&v[16 * c]);
+      for (int k = 0; k < 4; ++k) tmem_ld16(sa + 16 * k, (uint32_t*)&v[16 * k]);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(s_read_b + 8 * kb);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
       if (issuer) bulk_wait_read_all();                  // the previous copy has left the staging buffer
       named_bar_sync(2, 128);
       // the partial goes out in f16 (half the distributed-shared-memory bytes of fp32; the
       // partial scores stay far inside f16's range and its 11-bit significand costs the
       // scores ~1e-3 relative, well inside the output tolerance)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // chunk c (8 values) of row h at slot c ^ (h & 7): no bank conflicts
+      for (int k = 0; k < 8; ++k) {  // chunk k (8 values) of row h at slot k ^ (h & 7): no bank conflicts
         uint32_t w[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          __half2 hv = __floats2half2_rn(v[8 * c + 2 * j], v[8 * c + 2 * j + 1]);
+          __half2 hv = __floats2half2_rn(v[8 * k + 2 * j], v[8 * k + 2 * j + 1]);
           w[j] = *reinterpret_cast<uint32_t*>(&hv);
         }
-        stg_row[c ^ (h & 7)] = make_uint4(w[0], w[1], w[2], w[3]);
+        stg_row[k ^ (h & 7)] = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       named_bar_sync(2, 128);
       if (issuer) {
-        // the peer has consumed what we sent for tile k - 2 into the same buffer
-        const int xb = k & 1;
-        bool ok = mbar_wait_cluster(x_free_b + 8 * xb, ((k >> 1) & 1) ^ 1, abort_word, a.flag);
-        if (ok) {
+        // the peer's P.V(i - 2) has released the buffer we send into
+        const int xb = i & 1;
+        if (mbar_wait_cluster(x_free_b + 8 * xb, ((i >> 1) & 1) ^ 1, abort_word, a.flag)) {
           bulk_copy_to_peer(peer_x + xb * 16384, stg_s, 16384, peer_x_full + 8 * xb);
           bulk_commit_group();
         }
@@ -292,72 +365,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     }
     if (issuer) bulk_wait_read_all();
   } else {
-    // ---------------- softmax: thread h <-> head h <-> TMEM lane h ----------------
-    const int h = threadIdx.x;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    // Q latent half of head h -> TMEM (bf16 pairs), zero for padding heads
-    {
-      const uint4* src = (const uint4*)(a.q_abs + ((long long)b * a.H + (h < a.H ? h : 0)) * 512 + r * 256);
+    // ---------------- softmax: head h <-> TMEM lane h, columns [32 g, 32 g + 32) of each tile ----------------
+    const int q = warp & 3, g = warp >> 2;
+    const int h = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    // this half's share of sequence b's query: 128 latent values of CTA r's half
+    // -> TMEM columns [64 g, 64 g + 64), 32 rotary values -> [128 + 16 g, 128 + 16 g + 16)
+    auto load_q = [&](int b) {
+      const bool live = h < a.H;
+      const long long qh = (long long)b * a.H + (live ? h : 0);
+      const uint4* src = (const uint4*)(a.q_abs + qh * 512 + r * 256 + 128 * g);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t q[16];
+      for (int k4 = 0; k4 < 4; ++k4) {
+        uint32_t qv[16];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint4 v = (h < a.H) ? src[4 * c + k] : make_uint4(0, 0, 0, 0);
-          q[4 * k] = v.x; q[4 * k + 1] = v.y; q[4 * k + 2] = v.z; q[4 * k + 3] = v.w;
+          const uint4 v = live ? src[4 * k4 + k] : make_uint4(0, 0, 0, 0);
+          qv[4 * k] = v.x; qv[4 * k + 1] = v.y; qv[4 * k + 2] = v.z; qv[4 * k + 3] = v.w;
         }
-        tmem_st16(tmem + ATT_TM_Q + lane_base + 16 * c, q);
+        tmem_st16(tmem + ATT_TM_Q + lane_base + 64 * g + 16 * k4, qv);
       }
+      const uint4* pe = (const uint4*)(a.q_pe + qh * 64 + 32 * g);
+      uint32_t pv[16];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint4 v = live ? pe[k] : make_uint4(0, 0, 0, 0);
+        pv[4 * k] = v.x; pv[4 * k + 1] = v.y; pv[4 * k + 2] = v.z; pv[4 * k + 3] = v.w;
+      }
+      tmem_st16(tmem + ATT_TM_QPE + lane_base + 16 * g, pv);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(q_ready);
-    }
-    const uint32_t peer_x_free = mapa_shared(x_free_b, peer);
-    // block of tile t, loaded one tile ahead (only its validity is needed here)
-    auto tile_block = [&](int t) -> int {
-      return t < T ? a.block_table[(long long)b * a.mbps + (r0 + 64 * t) / a.bs] : 0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
     };
-    int blk_next = tile_block(0);
+    TileWalk w{pref, a.n, 0, 0};
+    w.start(g0);
+    load_q(w.b);
+    // block of tile i + 1, loaded one tile ahead (only its validity is needed here)
+    auto tile_block = [&](const TileWalk& t) { return a.block_table[(long long)t.b * a.mbps + (64 * t.lt) / a.bs]; };
+    int blk_next = tile_block(w);
+    int seq_len = attn_seq_len(a, w.b);
     float m_ref = -INFINITY, l = 0.f;
+    int tseg = 0, kseg = 0;   // tile within the segment, segments done
     bool ok = true;
-    for (int t = 0; t < T && ok; ++t) {
-      const int sb = t & 1, st = t % ATT_NST;
+    for (int i = 0; i < N && ok; ++i, w.next()) {
+      const int b = w.b, lt = w.lt, st = i % ATT_NST, xb = i & 1;
+      const bool last = (i == N - 1 || w.seg_last());
       const int blk = blk_next;
-      blk_next = tile_block(t + 1);
-      const int valid = (blk >= 0 && blk < a.n_blocks) ? min(64, r1 - (r0 + 64 * t)) : 0;
-      const int xb = t & 1;
-      if (h == 0) mbar_arrive_expect_tx(x_full_b + 8 * xb, 16384);
-      if (!mbar_wait_warp(x_full_b + 8 * xb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      if (!mbar_wait_warp(s_full_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (i + 1 < N) {
+        TileWalk wn = w;
+        wn.next();
+        blk_next = tile_block(wn);
+      }
+      const int valid = (blk >= 0 && blk < a.n_blocks) ? min(64, seq_len - 64 * lt) : 0;
+      if (threadIdx.x == 0) mbar_arrive_expect_tx(x_full_b + 8 * xb, 16384);
+      if (!mbar_wait_warp(s_full, i & 1, abort_word, a.flag)) { ok = false; break; }
       tc_fence_after();
-      float v[64];
-      const uint32_t sp_addr = tmem + ATT_TM_S + 64 * sb + lane_base;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld16(sp_addr + 16 * c, (uint32_t*)&v[16 * c]);
+      float v[32];
+      const uint32_t sp_addr = tmem + ATT_TM_S + 32 * g + lane_base;
+      tmem_ld16(sp_addr, (uint32_t*)&v[0]);
+      tmem_ld16(sp_addr + 16, (uint32_t*)&v[16]);
       tmem_ld_wait();
-      const uint4* xloc = (const uint4*)(smem + SM::X_OFF + xb * 16384 + h * 128);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);   // the next S may overwrite the buffer
+      if (!mbar_wait_warp(x_full_b + 8 * xb, (i >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      // row h, chunks 4 g .. 4 g + 3 of the peer's partial; P(i) later goes to exactly these bytes
+      uint4* xrow = (uint4*)(smem + SM::X_OFF + xb * 16384 + h * 128);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 x = xloc[c ^ (h & 7)];
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      for (int k = 0; k < 4; ++k) {
+        const uint4 x = xrow[(4 * g + k) ^ (h & 7)];
+        const uint32_t wx[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
-          v[8 * c + 2 * j] += f.x;
-          v[8 * c + 2 * j + 1] += f.y;
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wx[j]));
+          v[8 * k + 2 * j] += f.x;
+          v[8 * k + 2 * j + 1] += f.y;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote_relaxed(peer_x_free + 8 * xb);
-      // online softmax in log2 units with a lazily moved reference max
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (valid < 64) {
+        const int vc = valid - 32 * g;   // valid columns of this half
 #pragma unroll
-        for (int j = 0; j < 64; ++j) v[j] = (j < valid) ? v[j] : -INFINITY;   // also drops NaN past the context
+        for (int j = 0; j < 32; ++j) v[j] = (j < vc) ? v[j] : -INFINITY;   // also drops NaN past the context
       }
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < 64; ++j) m4[j & 3] = fmaxf(m4[j & 3], v[j]);
-      const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.scale_log2;
+      for (int j = 0; j < 32; ++j) m4[j & 3] = fmaxf(m4[j & 3], v[j]);
+      const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      // the two halves of head h meet: both then take the same decisions
+      red[(xb * 2 + g) * 128 + h] = mloc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xch_b + 8 * (2 * q + xb));
+      if (!mbar_wait_warp(xch_b + 8 * (2 * q + xb), (i >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      const float mt = fmaxf(mloc, red[(xb * 2 + (g ^ 1)) * 128 + h]) * a.scale_log2;
+      // online softmax in log2 units with a lazily moved reference max
       float alpha = 1.f;
       bool rescale = false;
       if (mt > m_ref + 8.f) {
@@ -366,74 +467,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       }
       const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int j = 0; j < 64; j += 2) {
+      for (int j = 0; j < 32; j += 2) {
         const float e0 = ex2_approx(fmaf(v[j], a.scale_log2, nm)), e1 = ex2_approx(fmaf(v[j + 1], a.scale_log2, nm));
         __nv_bfloat162 pb = __floats2bfloat162_rn(e0, e1);
         ps[(j >> 1) & 3] += e0 + e1;
         pk[j >> 1] = *reinterpret_cast<uint32_t*>(&pb);
       }
       const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      if (__any_sync(0xffffffffu, rescale) && t >= 1) {
-        // P.V of the previous tiles must be complete before O is touched
-        if (!mbar_wait_warp(o_done, (t - 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (__any_sync(0xffffffffu, rescale) && tseg >= 1) {
+        // P.V(i - 2) is complete (its release let the peer fill this X buffer), so
+        // waiting for the phase of P.V(i - 1) cannot pass early; O must not be
+        // touched before it completes
+        if (!mbar_wait_warp(o_done, (i - 1) & 1, abort_word, a.flag)) { ok = false; break; }
         tc_fence_after();
-        for (int c = 0; c < 16; ++c) {
+        for (int k = 0; k < 8; ++k) {
           uint32_t o[16];
-          tmem_ld16(tmem + ATT_TM_O + lane_base + 16 * c, o);
+          const uint32_t oa = tmem + ATT_TM_O + lane_base + 128 * g + 16 * k;
+          tmem_ld16(oa, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st16(tmem + ATT_TM_O + lane_base + 16 * c, o);
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st16(oa, o);
         }
+        tmem_st_wait();
+        tc_fence_before();
       }
       l = l * alpha + psum;
       if (valid < 64) {
         // rows past the context may hold anything (even NaN); P is 0 there, but
         // 0 * NaN is not, so clear them in the four latent slots before P.V
-        // latent rows are laid out [8 row octets][4 k-blocks][8 rows][128 B]
-        uint8_t* tl = smem + SM::TILE_OFF + st * SM::STAGE;
-        for (int row = valid + (h >> 1); row < 64; row += 64) {
-          uint8_t* rp = tl + (row >> 3) * 4096 + (row & 7) * 128 + (h & 1) * 2048;
+        // (latent rows are laid out [8 row octets][4 k-blocks][8 rows][128 B])
+        const int ti = g * 128 + h, row = valid + (ti >> 2);
+        if (row < 64) {
+          uint8_t* rp = smem + SM::TILE_OFF + st * SM::STAGE + (row >> 3) * 4096 + (ti & 3) * 1024 + (row & 7) * 128;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)   // two of the four k-blocks: 256 bytes
-            *reinterpret_cast<uint4*>(rp + (c >> 3) * 1024 + 16 * (c & 7)) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-      }
-      // the sender must have read S(t) before P overwrites it
-      if (!mbar_wait_warp(s_read_b + 8 * sb, (t >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
-      tmem_st16(sp_addr, pk);            // P over S: 32 columns of bf16 pairs
-      tmem_st16(sp_addr + 16, pk + 16);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_full_b + 8 * sb);
-    }
-    // every MMA, the last P.V included, has completed once `fin` does (waiting
-    // on o_done's parity could pass while an earlier P.V is still running)
-    if (ok && mbar_wait_warp(fin, 0, abort_word, a.flag)) {
-      tc_fence_after();
-      float* po = a.part_o + (unit * a.H + h) * 512 + r * 256;
-      for (int c = 0; c < 16; ++c) {
-        uint32_t o[16];
-        tmem_ld16(tmem + ATT_TM_O + lane_base + 16 * c, o);
-        tmem_ld_wait();
-        if (h < a.H) {
-#pragma unroll
-          for (int k = 0; k < 16; k += 4)
-            *reinterpret_cast<float4*>(po + 16 * c + k) =
-                make_float4(__uint_as_float(o[k]), __uint_as_float(o[k + 1]), __uint_as_float(o[k + 2]),
-                            __uint_as_float(o[k + 3]));
+          for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(rp + 16 * k) = make_uint4(0, 0, 0, 0);
         }
       }
-      if (h < a.H) {
-        ml[(unit * a.H + h) * 2] = m_ref * 0.69314718055994531f;   // natural-log units
-        ml[(unit * a.H + h) * 2 + 1] = l;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        xrow[(4 * g + k) ^ (h & 7)] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full_b + 8 * xb);
+      ++tseg;
+      if (last) {
+        // the segment's S MMAs are all complete (the softmax read each S): the next
+        // segment's query may replace this one while the last P.V runs
+        if (i + 1 < N) {
+          TileWalk wn = w;
+          wn.next();
+          load_q(wn.b);
+          seq_len = attn_seq_len(a, wn.b);
+        }
+        const int j = c - pref[b] / per;               // this segment's split slot in sequence b
+        const long long unit = (long long)b * a.splits + j;
+        float* const ml = a.part_ml + r * a.ml_r;      // this CTA's (m, l) copy
+        if (!mbar_wait_warp(o_seg, kseg & 1, abort_word, a.flag)) { ok = false; break; }
+        tc_fence_after();
+        float* po = a.part_o + (unit * a.H + h) * 512 + r * 256 + 128 * g;
+        for (int k = 0; k < 8; ++k) {
+          uint32_t o[16];
+          tmem_ld16(tmem + ATT_TM_O + lane_base + 128 * g + 16 * k, o);
+          tmem_ld_wait();
+          if (h < a.H) {
+#pragma unroll
+            for (int jj = 0; jj < 16; jj += 4)
+              *reinterpret_cast<float4*>(po + 16 * k + jj) =
+                  make_float4(__uint_as_float(o[jj]), __uint_as_float(o[jj + 1]), __uint_as_float(o[jj + 2]),
+                              __uint_as_float(o[jj + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free);   // the next segment's first P.V may overwrite O
+        // the row sum is the two halves' sums
+        if (g == 1) {
+          red_l[h] = l;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(l_done + 8 * q);
+        } else if (mbar_wait_warp(l_done + 8 * q, kseg & 1, abort_word, a.flag)) {
+          if (h < a.H) {
+            ml[(unit * a.H + h) * 2] = m_ref * 0.69314718055994531f;   // natural-log units
+            ml[(unit * a.H + h) * 2 + 1] = l + red_l[h];
+          }
+        } else {
+          ok = false;
+          break;
+        }
+        m_ref = -INFINITY;
+        l = 0.f;
+        tseg = 0;
+        ++kseg;
       }
-    } else if (h < a.H) {
-      ml[(unit * a.H + h) * 2] = -INFINITY;
-      ml[(unit * a.H + h) * 2 + 1] = 0.f;
     }
   }
   tc_fence_before();

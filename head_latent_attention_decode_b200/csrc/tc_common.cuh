@@ -377,3 +377,19 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar)
 
 }  // namespace tc
 }  // namespace mla
+
+namespace mla {
+namespace tc {
+
+// Arrive once on the mbarrier at shared-memory offset `bar` of every CTA of the
+// cluster in `cta_mask` when all previously issued tcgen05.mma of this thread
+// complete (a commit signal, not a data load).
+__device__ __forceinline__ void mma_commit_cta_mask(uint32_t bar, uint16_t cta_mask) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   bar),
+               "h"(cta_mask)
+               : "memory");
+}
+
+}  // namespace tc
+}  // namespace mla

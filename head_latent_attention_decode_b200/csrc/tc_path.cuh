@@ -655,7 +655,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
 static inline int tc_attention_core(const mla_handle* h, const void* q_abs, const void* q_pe, const void* kv_cache,
                                     int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
                                     int max_ctx, int n, float* part_o, float* part_ml, int splits, bf16* o_lat,
-                                    int* flag, cudaStream_t s) {
+                                    int* flag, int* nseg, cudaStream_t s) {
   const mla_config& c = h->cfg;
   const TcState& T = h->tc;
   const int H = c.n_heads, dr = c.qk_rope, rkv = c.kv_lora_rank;
@@ -665,6 +665,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
   const float* sink = h->has_sink ? (const float*)(h->base + h->L.sink) : nullptr;
   long long ml_r = 0;         // offset of the second CTA's (m, l) copy (tensor-core kernels)
   int half_cols = 0;          // latent columns per (m, l) copy (0: one copy)
+  int* seg_counts = nullptr;  // split partials per sequence, when a kernel reports them
   const bool latent_ok = rkv == 512 && dr == 64 && c.block_size % 64 == 0 && (((uintptr_t)q_abs) & 15) == 0 &&
                          (((uintptr_t)q_pe) & 15) == 0;
   if (latent_ok && H <= 32) {
@@ -721,31 +722,29 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     }
     mla_timer_end("attn", s);
     mla_count_launch(1);
-  } else if (latent_ok && H <= 128) {
-    // (sequence, split) clusters: about three waves of CTA pairs, at most the
-    // splits the workspace holds (six waves balanced random context lengths
-    // better, but the merge's re-read of the extra partials cost as much)
+  } else if (latent_ok && H <= 128 && n <= ATT_MAX_SEQ && splits >= 2) {
+    // persistent and balanced: one 2-CTA cluster per SM pair, each an equal
+    // slice of the batch's 64-row tiles; a slice holds at least `min_per` tiles
+    // so that no sequence spreads over more segments than the workspace holds
     const int pairs = T.num_sms / 2 > 0 ? T.num_sms / 2 : 74;
-    int sp = (int)cdiv(3 * pairs, n);
-    if (sp > splits) sp = splits;
-    if (sp < 1) sp = 1;
-    const int chunk = (int)cdiv(cdiv(max_ctx, sp), 64) * 64;
-    sp = (int)cdiv(max_ctx, chunk);
-    splits = sp;
-    CUtensorMap mqp, mc, ml;
-    if ((st = make_map2(&mqp, q_pe, dr, (long long)n * H, dr, 128)) != MLA_OK) return st;
+    const int max_tiles = (int)cdiv(max_ctx, 64);
+    CUtensorMap mc, ml;
     if ((st = make_map2(&mc, kv_cache, R, (long long)n_blocks * c.block_size, R, 64)) != MLA_OK) return st;
     if ((st = make_map_cache_groups(&ml, kv_cache, R, (long long)n_blocks * c.block_size, 4)) != MLA_OK) return st;
     TcAttnArgs ta{};
-    ta.n = n; ta.H = H; ta.splits = sp; ta.chunk = chunk;
+    ta.n = n; ta.H = H; ta.splits = splits; ta.chunk = 0;
     ta.bs = c.block_size; ta.n_blocks = n_blocks; ta.mbps = mbps; ta.max_ctx = max_ctx;
-    ta.block_table = block_table; ta.ctx = ctx; ta.q_abs = (const bf16*)q_abs;
+    ta.block_table = block_table; ta.ctx = ctx; ta.q_abs = (const bf16*)q_abs; ta.q_pe = (const bf16*)q_pe;
     ta.lat_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? 0 : dr;
     ta.rope_col0 = c.row_layout == MLA_ROW_LATENT_FIRST ? rkv : 0;
     ta.scale_log2 = h->scale * 1.4426950408889634f;
     ta.part_o = part_o; ta.part_ml = part_ml; ta.flag = flag;
-    ta.ml_r = ml_r = (long long)n * sp * H * 2;
+    ta.ml_r = ml_r = (long long)n * splits * H * 2;
+    ta.units = pairs;
+    ta.min_per = (int)cdiv(max_tiles, splits - 1);
+    ta.nseg = nseg;
     half_cols = 256;
+    seg_counts = nseg;
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -754,7 +753,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
       attr[dev] = true;
     }
     mla_timer_begin("attn", s);
-    launch_pdl(tc_attn_decode_kernel, 2 * n * sp, ATT_THREADS, AttnSmem::SIZE, s, mqp, mc, ml, ta);
+    launch_pdl(tc_attn_decode_kernel, 2 * pairs, ATT_THREADS, AttnSmem::SIZE, s, mc, ml, ta);
     mla_timer_end("attn", s);
     mla_count_launch(1);
   } else {
@@ -772,7 +771,7 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     mla_count_launch(1);
   }
   launch_pdl(attn_combine_kernel<bf16>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits, H,
-             rkv, o_lat, sink, ml_r, half_cols);
+             rkv, o_lat, sink, ml_r, half_cols, (const int*)seg_counts);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -780,7 +779,8 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
 static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const void* q_pe, const void* kv_cache,
                                  int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
                                  int max_ctx, int n, void* out, void* head, char* ws, size_t tc_off,
-                                 cudaStream_t s, float* part_o, float* part_ml, int splits, bf16* o_lat) {
+                                 cudaStream_t s, float* part_o, float* part_ml, int splits, bf16* o_lat,
+                                 int* nseg) {
   const mla_config& c = h->cfg;
   const TcDecodeWs W = tc_decode_ws(h, n);
   char* tw = ws + tc_off;
@@ -788,7 +788,7 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   const int H = c.n_heads, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
   const int bn = pick_bn(n);
   int st = tc_attention_core(h, q_abs, q_pe, kv_cache, n_blocks, block_table, mbps, ctx, max_ctx, n, part_o,
-                             part_ml, splits, o_lat, flag, s);
+                             part_ml, splits, o_lat, flag, nseg, s);
   if (st != MLA_OK) return st;
   // 2. head_out[h] = o_lat[h] @ W_UV[h]  (A = Wuv[h] [d_v, r_kv], B = o_lat[:, h, :])
   void* f16buf = tw + W.bf16c;
