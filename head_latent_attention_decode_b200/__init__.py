@@ -47,13 +47,13 @@ class mla_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "hidden", "n_heads", "q_lora_rank", "kv_lora_rank", "qk_nope", "qk_rope", "v_dim",
         "block_size")] + [("norm_eps", ctypes.c_float), ("softmax_scale", ctypes.c_float)] + [
-        (n, ctypes.c_int) for n in ("act_dtype", "weight_dtype", "row_layout")]
+        (n, ctypes.c_int) for n in ("act_dtype", "weight_dtype", "row_layout", "o_groups", "o_lora_rank")]
 
 
 class mla_weights_desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "wq_a", "wq_b", "wkv_a", "wkv_b", "wo", "q_norm_w", "kv_norm_w", "wq_a_scale",
-        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale", "attn_sink")]
+        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale", "attn_sink", "wo_a", "wo_b")]
 
 
 class MlaError(RuntimeError):
@@ -153,7 +153,7 @@ def make_config(shape, row_layout: int = MLA_ROW_LATENT_FIRST, softmax_scale: fl
     return mla_config(shape.hidden, shape.n_heads, shape.q_lora_rank, shape.kv_lora_rank,
                       shape.qk_nope, shape.qk_rope, shape.v_dim, shape.block_size,
                       shape.norm_eps, softmax_scale, dt[shape.act_dtype], dt[shape.weight_dtype],
-                      row_layout)
+                      row_layout, getattr(shape, "o_groups", 0), getattr(shape, "o_lora_rank", 0))
 
 
 def mla_weights_bytes(cfg: mla_config) -> int:
@@ -161,11 +161,11 @@ def mla_weights_bytes(cfg: mla_config) -> int:
 
 
 def mla_init_weights(cfg: mla_config, weights: dict, dst: torch.Tensor, stream=None) -> int:
-    """weights: name -> device tensor (wq_a, wq_b, wkv_a, wkv_b, wo, q_norm_w, kv_norm_w,
-    *_scale for FP8, optional attn_sink [H] fp32). Returns the opaque handle (int)."""
+    """weights: name -> device tensor (wq_a, wq_b, wkv_a, wkv_b, wo or wo_a + wo_b, q_norm_w,
+    kv_norm_w, *_scale for FP8, optional attn_sink [H] fp32). Returns the opaque handle (int)."""
     d = mla_weights_desc(*[_ptr(weights.get(n)) for n in (
         "wq_a", "wq_b", "wkv_a", "wkv_b", "wo", "q_norm_w", "kv_norm_w", "wq_a_scale",
-        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale", "attn_sink")])
+        "wq_b_scale", "wkv_a_scale", "wkv_b_scale", "wo_scale", "attn_sink", "wo_a", "wo_b")])
     h = ctypes.c_void_p()
     _check(lib().mla_init_weights(ctypes.byref(cfg), ctypes.byref(d), _ptr(dst), _nbytes(dst),
                                   _stream(stream), ctypes.byref(h)), "mla_init_weights")

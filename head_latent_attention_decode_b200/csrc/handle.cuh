@@ -28,13 +28,16 @@ void mla_timer_end(const char* kernel, cudaStream_t s);
 //   Wuk  [H][r_kv][d_n]   Wuk[h][c][p] = wkv_b[c][h*(d_n+d_v) + p]
 //   Wuv  [H][d_v][r_kv]   Wuv[h][d][c] = wkv_b[c][h*(d_n+d_v) + d_n + d]
 //   Wkvb [H*(d_n+d_v), r_kv]                          (prefill)
-//   Wo   [D, H*d_v]
+//   Wo   [D, H*d_v]                                   (dense output projection)
+//   Woa  [G][r_o][(H/G)*d_v]  Woa[g][j][i] = wo_a[g*(H/G)*d_v + i][j]   (grouped, o_lora_rank > 0)
+//   Wob  [D, G*r_o]
 // FP8 blobs add fp32 scales per 128x128 block of each K-major matrix,
 // [ceil(N/128)][ceil(K/128)].
 struct WeightLayout {
   int Nq1, N1, R, Hq, Hkv;
   size_t esz;
-  size_t W1, Wqb, Wuk, Wuv, Wkvb, Wo, gq, gkv, sink;
+  size_t W1, Wqb, Wuk, Wuv, Wkvb, Wo, Woa, Wob, gq, gkv, sink;
+  int G, ro, Kg;   // grouped output projection: groups, low rank, inputs per group (0 = dense wo)
   size_t sW1, sWqb, sWuk, sWuv, sWkvb, sWo;
   size_t total;
 };

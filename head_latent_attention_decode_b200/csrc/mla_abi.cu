@@ -61,6 +61,13 @@ static int validate_config(const mla_config* c) {
     if (c->q_lora_rank % 128 || c->qk_nope % 128 || c->v_dim % 128 || Hq % 128)
       return MLA_ERR_UNSUPPORTED;
   }
+  // grouped low-rank output projection
+  if (c->o_lora_rank < 0 || c->o_groups < 0) return MLA_ERR_INVALID_ARG;
+  if (c->o_lora_rank > 0) {
+    if (c->o_groups < 1 || c->n_heads % c->o_groups) return MLA_ERR_INVALID_ARG;
+    if (c->weight_dtype == MLA_FP8_E4M3_B128) return MLA_ERR_UNSUPPORTED;
+    if (c->o_lora_rank % 64 || ((long long)(c->n_heads / c->o_groups) * c->v_dim) % 64) return MLA_ERR_UNSUPPORTED;
+  }
   return MLA_OK;
 }
 
@@ -85,7 +92,15 @@ static WeightLayout make_layout(const mla_config* c) {
   L.Wuk = put((size_t)H * rkv * dn * L.esz);
   L.Wuv = put((size_t)H * dv * rkv * L.esz);
   L.Wkvb = put((size_t)L.Hkv * rkv * L.esz);
-  L.Wo = put((size_t)D * H * dv * L.esz);
+  if (c->o_lora_rank > 0) {
+    L.G = c->o_groups;
+    L.ro = c->o_lora_rank;
+    L.Kg = H / L.G * dv;
+    L.Woa = put((size_t)L.G * L.ro * L.Kg * L.esz);
+    L.Wob = put((size_t)D * L.G * L.ro * L.esz);
+  } else {
+    L.Wo = put((size_t)D * H * dv * L.esz);
+  }
   L.gq = rq ? put((size_t)rq * 4) : 0;
   L.gkv = put((size_t)rkv * 4);
   L.sink = put((size_t)H * 4);
@@ -107,8 +122,8 @@ static WeightLayout make_layout(const mla_config* c) {
 // [0, 256): device flag (int32 at 0) and counters. Then decode and prefill
 // scratch share one region (calls on one workspace are stream-ordered).
 struct WsLayout {
-  size_t Y1, qn, Q, part_o, part_ml, nseg, o_lat, head, xn;   // decode
-  size_t pY1, pqn, pQ, pcn, pkpe, pKV, phead, pDQ;             // prefill
+  size_t Y1, qn, Q, part_o, part_ml, nseg, o_lat, head, xn, oy;   // decode
+  size_t pY1, pqn, pQ, pcn, pkpe, pKV, phead, pDQ, poy;            // prefill
   size_t tc;                                                   // tensor-core path scratch
   size_t dec_total;                                            // what the decode calls need
   size_t total;                                                // what every call needs
@@ -138,6 +153,7 @@ static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
   W.o_lat = put((size_t)n * H * rkv * a);
   W.head = put((size_t)n * H * dv * a);
   W.xn = put((size_t)n * c->hidden * a);
+  W.oy = put((size_t)n * (L.G ? L.G * L.ro : 1) * a);   // grouped output projection: the low-rank rows
   W.tc = put(tc_decode_ws_bytes(h, n, max_ctx));
   const size_t dec_end = off;
   W.dec_total = dec_end;
@@ -149,6 +165,7 @@ static WsLayout make_ws(const mla_handle* h, long long n, int max_ctx) {
   W.pkpe = put((size_t)n * dr * a);
   W.pKV = put((size_t)n * L.Hkv * a);
   W.phead = put((size_t)n * H * dv * a);
+  W.poy = put((size_t)n * (L.G ? L.G * L.ro : 1) * a);
   W.pDQ = put(tc_prefill_dequant_bytes(h));   // FP8 weights: one dequantised weight at a time
   W.total = dec_end > off ? dec_end : off;
   return W;
@@ -204,6 +221,27 @@ static LinearArgs lin(const void* A, long long lda, const void* W, long long ldw
   return a;
 }
 
+static void launch_o_proj_simt(const mla_handle* h, const void* head, void* out, void* y, long long n, cudaStream_t s) {
+  const WeightLayout& L = h->L;
+  const mla_config* c = &h->cfg;
+  const int H = c->n_heads, dv = c->v_dim, D = c->hidden;
+  const int ta = h->cfg.act_dtype == MLA_F32 ? 0 : 1;
+  const int tw = h->cfg.weight_dtype == MLA_F32 ? 0 : (h->cfg.weight_dtype == MLA_BF16 ? 1 : 2);
+  if (!L.G) {
+    const float* sc = L.sWo ? (const float*)(h->base + L.sWo) : nullptr;
+    launch_linear(ta, tw, ta, lin(head, (long long)H * dv, h->base + L.Wo, (long long)H * dv, sc,
+                                  cdiv((long long)H * dv, 128), out, D, (int)n, D, H * dv), 1, s);
+    return;
+  }
+  // y[:, g*r_o + j] = head[:, g*Kg .. (g+1)*Kg) @ wo_a block g; then out = y @ wo_b
+  LinearArgs a = lin(head, (long long)H * dv, h->base + L.Woa, L.Kg, nullptr, 0, y, (long long)L.G * L.ro,
+                     (int)n, L.ro, L.Kg);
+  a.a_batch = L.Kg; a.w_batch = (long long)L.ro * L.Kg; a.c_batch = L.ro; a.s_batch = 0;
+  launch_linear(ta, tw, ta, a, L.G, s);
+  launch_linear(ta, tw, ta, lin(y, (long long)L.G * L.ro, h->base + L.Wob, (long long)L.G * L.ro, nullptr, 0, out, D,
+                                (int)n, D, L.G * L.ro), 1, s);
+}
+
 template <typename K>
 static void set_smem(K kernel, size_t bytes) {
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -216,6 +254,11 @@ static int wcode(const mla_handle* h) {
   return h->cfg.weight_dtype == MLA_F32 ? 0 : (h->cfg.weight_dtype == MLA_BF16 ? 1 : 2);
 }
 static int acode(const mla_handle* h) { return h->cfg.act_dtype == MLA_F32 ? 0 : 1; }
+
+// out [n, D] = the output projection of head [n, H*d_v] on CUDA cores: the dense
+// wo, or the grouped low-rank wo_a (one batched product per group of heads, into
+// y [n, G*r_o] in act dtype) then wo_b ("Struct MlaWeights", wo_a / wo_b).
+static void launch_o_proj_simt(const mla_handle* h, const void* head, void* out, void* y, long long n, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // entry points
@@ -268,7 +311,8 @@ int mla_init_weights(const mla_config* cfg, const mla_weights_desc* w, void* dst
   if (((uintptr_t)dst) % 256) return MLA_ERR_INVALID_ARG;
   const bool fp8 = cfg->weight_dtype == MLA_FP8_E4M3_B128;
   const int rq = cfg->q_lora_rank;
-  if (!w->wq_b || !w->wkv_a || !w->wkv_b || !w->wo || !w->kv_norm_w) return MLA_ERR_INVALID_ARG;
+  if (!w->wq_b || !w->wkv_a || !w->wkv_b || !w->kv_norm_w) return MLA_ERR_INVALID_ARG;
+  if (cfg->o_lora_rank > 0 ? (!w->wo_a || !w->wo_b) : !w->wo) return MLA_ERR_INVALID_ARG;
   if (rq && (!w->wq_a || !w->q_norm_w)) return MLA_ERR_INVALID_ARG;
   if (fp8 && (!w->wq_b_scale || !w->wkv_a_scale || !w->wkv_b_scale || !w->wo_scale || (rq && !w->wq_a_scale)))
     return MLA_ERR_INVALID_ARG;
@@ -303,7 +347,13 @@ int mla_init_weights(const mla_config* cfg, const mla_weights_desc* w, void* dst
   gather(L.Wuk, w->wkv_b, 0, dn + dv, ldkvb, 1, H, rkv, dn, e);
   gather(L.Wuv, w->wkv_b, dn, dn + dv, 1, ldkvb, H, dv, rkv, e);
   gather(L.Wkvb, w->wkv_b, 0, 0, 1, ldkvb, 1, L.Hkv, rkv, e);
-  gather(L.Wo, w->wo, 0, 0, 1, D, 1, D, H * dv, e);
+  if (L.G) {
+    // Woa[g][j][i] = wo_a[g*Kg + i][j]; Wob[d][k] = wo_b[k][d]
+    gather(L.Woa, w->wo_a, 0, (long long)L.Kg * L.ro, 1, L.ro, L.G, L.ro, L.Kg, e);
+    gather(L.Wob, w->wo_b, 0, 0, 1, D, 1, D, L.G * L.ro, e);
+  } else {
+    gather(L.Wo, w->wo, 0, 0, 1, D, 1, D, H * dv, e);
+  }
   if (rq) cudaMemcpyAsync(h->base + L.gq, w->q_norm_w, (size_t)rq * 4, cudaMemcpyDeviceToDevice, s);
   cudaMemcpyAsync(h->base + L.gkv, w->kv_norm_w, (size_t)rkv * 4, cudaMemcpyDeviceToDevice, s);
   h->has_sink = w->attn_sink != nullptr;
@@ -465,7 +515,7 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
   char* wsb = (char*)ws;
   int* flag = (int*)wsb;
   const WeightLayout& L = h->L;
-  const int H = c->n_heads, dr = c->qk_rope, rkv = c->kv_lora_rank, dv = c->v_dim, D = c->hidden;
+  const int H = c->n_heads, dr = c->qk_rope, rkv = c->kv_lora_rank, dv = c->v_dim;
   const int ta = acode(h), tw = wcode(h);
   void* head = head_out ? head_out : (void*)(wsb + W.head);
   if (tc_decode_attn_supported(h, n, max_context_len)) {
@@ -510,9 +560,8 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
                      (long long)H * dv, n, dv, rkv);
   a.a_batch = rkv; a.w_batch = (long long)dv * rkv; a.c_batch = dv; a.s_batch = cdiv(dv, 128) * cdiv(rkv, 128);
   launch_linear(ta, tw, ta, a, H, s);
-  // out = head_out @ wo
-  launch_linear(ta, tw, ta, lin(head, (long long)H * dv, h->base + L.Wo, (long long)H * dv, wscale(h, L.sWo),
-                                cdiv((long long)H * dv, 128), out, D, n, D, H * dv), 1, s);
+  // out = head_out @ wo (or wo_a -> wo_b)
+  launch_o_proj_simt(h, head, out, wsb + W.oy, n, s);
   return cuda_status();
 }
 
@@ -679,7 +728,7 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos, cons
   void* head = head_out ? head_out : (void*)(wsb + W.phead);
   if (tc_prefill_supported(h, S)) {
     const int r = tc_prefill(h, hidden, S, cos, sin, out, head, kv_cache, n_blocks, slot_mapping, wsb,
-                             W.pY1, W.pqn, W.pQ, W.pcn, W.pkpe, W.pKV, W.pDQ, s);
+                             W.pY1, W.pqn, W.pQ, W.pcn, W.pkpe, W.pKV, W.pDQ, W.poy, s);
     return r != MLA_OK ? r : cuda_status();
   }
   float* Y1 = (float*)(wsb + W.pY1);
@@ -727,8 +776,7 @@ int mla_prefill(mla_handle* h, const void* hidden, int S, const float* cos, cons
   else { set_smem(prefill_attn_simt_kernel<bf16>, smem); prefill_attn_simt_kernel<bf16><<<grid, 128, smem, s>>>(pa); }
   mla_timer_end("prefill_attn", s);
   count_launch();
-  launch_linear(ta, tw, ta, lin(head, (long long)H * dv, h->base + L.Wo, (long long)H * dv, wscale(h, L.sWo),
-                                cdiv((long long)H * dv, 128), out, D, S, D, H * dv), 1, s);
+  launch_o_proj_simt(h, head, out, wsb + W.poy, S, s);
   return cuda_status();
 }
 

@@ -104,6 +104,58 @@ __device__ __forceinline__ int attn_seq_len(const TcAttnArgs& a, int b) {
   return (L < 1 || L > a.max_ctx || L > a.mbps * a.bs) ? 0 : L;
 }
 
+// The balanced schedule of a persistent attention kernel: the prefix sum of
+// the batch's tiles of `tile_rows` rows, in shared memory (pref[b] = tiles of
+// sequences 0..b-1, n + 1 entries, n <= 256), and the slice [g0, g1) of the
+// flattened tile list that cluster c takes (slices of `per` tiles, at least
+// a.min_per). Block 0 of the grid writes each sequence's segment count to
+// a.nseg. Every thread of the CTA calls it; it ends with a __syncthreads.
+__device__ __forceinline__ void attn_schedule(const TcAttnArgs& a, int tile_rows, int* pref, int c, uint32_t r,
+                                              int warp, int lane, int* per_out, int* g0_out, int* g1_out) {
+  if (warp == 0) {
+    int cnt[8], sum = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int b = 8 * lane + k;
+      int T = 0;
+      if (b < a.n) {
+        const int L = attn_seq_len(a, b);
+        if (L == 0 && c == 0 && r == 0) set_flag(a.flag, MLA_FLAG_BAD_CONTEXT);
+        T = (L + tile_rows - 1) / tile_rows;
+      }
+      cnt[k] = T;
+      sum += T;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int b = 8 * lane + k;
+      if (b < a.n) pref[b] = run;
+      run += cnt[k];
+    }
+    if (lane == 31) pref[a.n] = incl;   // the batch's tile count
+  }
+  __syncthreads();
+  const int total = pref[a.n];
+  int per = (total + a.units - 1) / a.units;
+  if (per < a.min_per) per = a.min_per;
+  if (blockIdx.x == 0) {   // segments of each sequence, for the merge
+    for (int b = threadIdx.x; b < a.n; b += blockDim.x) {
+      const int T = pref[b + 1] - pref[b];
+      a.nseg[b] = T > 0 ? (pref[b] + T - 1) / per - pref[b] / per + 1 : 0;
+    }
+  }
+  *per_out = per;
+  *g0_out = c * per;
+  *g1_out = min(total, c * per + per);
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     tc_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_lat,
                           TcAttnArgs a) {
@@ -140,46 +192,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- the schedule: tile prefix over the batch, then this cluster's slice ----
-  if (warp == 0) {
-    int cnt[8], sum = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int b = 8 * lane + k;
-      int T = 0;
-      if (b < a.n) {
-        const int L = attn_seq_len(a, b);
-        if (L == 0 && c == 0 && r == 0) set_flag(a.flag, MLA_FLAG_BAD_CONTEXT);
-        T = (L + 63) / 64;
-      }
-      cnt[k] = T;
-      sum += T;
-    }
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - sum;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int b = 8 * lane + k;
-      if (b < a.n) pref[b] = run;
-      run += cnt[k];
-    }
-    if (lane == 31) pref[a.n] = incl;   // the batch's tile count
-  }
-  __syncthreads();
-  const int total = pref[a.n];
-  int per = (total + a.units - 1) / a.units;
-  if (per < a.min_per) per = a.min_per;
-  const int g0 = c * per, g1 = min(total, g0 + per);
-  if (blockIdx.x == 0) {   // segments of each sequence, for the merge
-    for (int b = threadIdx.x; b < a.n; b += blockDim.x) {
-      const int T = pref[b + 1] - pref[b];
-      a.nseg[b] = T > 0 ? (pref[b] + T - 1) / per - pref[b] / per + 1 : 0;
-    }
-  }
+  int per, g0, g1;
+  attn_schedule(a, 64, pref, c, r, warp, lane, &per, &g0, &g1);
   if (g0 >= g1) return;   // both CTAs of the cluster take this branch together
   const int N = g1 - g0;
 
@@ -211,18 +225,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 8) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (lane 0 issues; lane k holds the block id of tile i + k) ----------------
     if (lane == 0) {
       prefetch_tmap(&tm_cache);
       prefetch_tmap(&tm_lat);
-      TileWalk w{pref, a.n, 0, 0};
-      w.start(g0);
-      int i = 0;
-      for (; i < N; ++i, w.next()) {
-        const int st = i % ATT_NST;
-        if (!mbar_wait(empty_b + 8 * st, ((i / ATT_NST) & 1) ^ 1, abort_word, a.flag)) break;
+    }
+    TileWalk w{pref, a.n, 0, 0};
+    w.start(g0);
+    int i = 0, blkv = 0;
+    for (; i < N; ++i, w.next()) {
+      if ((i & 31) == 0) {   // the block ids of the next 32 tiles, loaded in parallel
+        TileWalk wk = w;
+        for (int k = 0; k < lane && i + k + 1 < N; ++k) wk.next();
+        blkv = (i + lane < N) ? a.block_table[(long long)wk.b * a.mbps + (64 * wk.lt) / a.bs] : 0;
+      }
+      const int blk = __shfl_sync(0xffffffffu, blkv, i & 31);
+      const int st = i % ATT_NST;
+      if (!mbar_wait_warp(empty_b + 8 * st, ((i / ATT_NST) & 1) ^ 1, abort_word, a.flag)) break;
+      if (lane == 0) {
         const int j0 = 64 * w.lt;
-        const int blk = a.block_table[(long long)w.b * a.mbps + j0 / a.bs];
         long long row = -64;
         if (blk >= 0 && blk < a.n_blocks) row = (long long)blk * a.bs + (j0 % a.bs);
         else if (r == 0) set_flag(a.flag, MLA_FLAG_BAD_BLOCK);
@@ -233,7 +254,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         tma_load_4d(dst, &tm_lat, full_b + 8 * st, 0, 0, a.lat_col0 / 64 + 4 * (int)r, (int)(row / 8));
         if (rope) tma_load_3d(dst + 4 * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
       }
-      // drain the loads still in flight
+    }
+    // drain the loads still in flight
+    if (lane == 0) {
       for (int u = (i > ATT_NST ? i - ATT_NST : 0); u < i; ++u) {
         const uint64_t t1 = global_timer_ns();
         while (!mbar_try_wait(full_b + 8 * (u % ATT_NST), (u / ATT_NST) & 1))

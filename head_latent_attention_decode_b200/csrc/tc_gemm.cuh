@@ -85,18 +85,31 @@ __device__ __forceinline__ void gemm_store(const GemmArgs& g, int m, int n0, int
       const int hd = g.dn + g.dr;
       const int h = m / hd, jj = m % hd;
       const bool odd = (m & 1) != 0;
+      const bool rot = m_ok && jj >= g.dn;
+      // The 16 tokens' cos / sin first: a load placed after a store to q (which may alias the
+      // tables, as far as the compiler knows) waits for it, and under a saturated memory system
+      // that wait is long.
+      float cs[16], sn[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int n = n0 + j;
+        cs[j] = sn[j] = 0.f;
+        if (rot && n < g.N) {
+          const long long t = (long long)n * (g.dr >> 1) + ((jj - g.dn) >> 1);
+          cs[j] = g.cos[t];
+          sn[j] = g.sin[t];
+        }
+      }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float v = __uint_as_float(r[j]);
         const float partner = __shfl_xor_sync(0xffffffffu, v, 1);   // all lanes take part
         const int n = n0 + j;
         if (!m_ok || n >= g.N) continue;
-        if (jj < g.dn) {
+        if (!rot) {
           ((bf16*)g.out)[((long long)n * g.H + h) * g.dn + jj] = __float2bfloat16_rn(v);
         } else {
-          const int i = (jj - g.dn) >> 1;
-          const float c = g.cos[(long long)n * (g.dr >> 1) + i], s = g.sin[(long long)n * (g.dr >> 1) + i];
-          const float o = odd ? (partner * s + v * c) : (v * c - partner * s);
+          const float o = odd ? (partner * sn[j] + v * cs[j]) : (v * cs[j] - partner * sn[j]);
           ((bf16*)g.out2)[((long long)n * g.H + h) * g.dr + (jj - g.dn)] = __float2bfloat16_rn(o);
         }
       }

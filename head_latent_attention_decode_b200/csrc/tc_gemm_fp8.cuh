@@ -5,12 +5,16 @@
 // A = the FP8 weight matrix (M = output features, 128 per tile = one scale row),
 // B = the tokens converted to f16 (N = BN; exact for |x| in f16's normal range,
 // which holds every activation of this layer). Per 128-wide K block:
-//   TMA brings the 128 x 128 code tile and the 2 x [BN x 64] f16 token tiles;
-//   warps 0-7 decode the codes to f16 with cvt.rn.f16x2.e4m3x2 (exact: every
-//   E4M3 value is an f16 value) into a 128-byte-swizzled tile;
-//   tcgen05 (kind::f16, f16 x f16 -> fp32) multiplies that block alone into one
-//   of two TMEM partials;
-//   warps 0-7 add scale * partial to fp32 registers (two column halves).
+//   TMA brings the 128 x 128 code tile into a deep ring of its own (the codes
+//   are the HBM stream) and the BN x 128 f16 token tile into a shorter one
+//   (the tokens come from L2);
+//   warps 0-3 decode the codes to f16 with cvt.rn.f16x2.e4m3x2 (exact: every
+//   E4M3 value is an f16 value) straight into TMEM, one weight row per thread,
+//   so the code stage is free again as soon as it is read;
+//   tcgen05 (kind::f16, A from TMEM, f16 x f16 -> fp32) multiplies that block
+//   alone into one of three TMEM partials;
+//   warps 4-11 add scale * partial to fp32 registers (two column halves);
+//   warp 12 issues the TMA loads, warp 13 the MMAs.
 // So the scale multiplies each block's exact fp32 partial sum, the same value
 // as dequantising every weight in fp32 before the MAC, up to fp32 rounding.
 // The epilogue modes are those of tc_gemm.cuh.
@@ -29,17 +33,24 @@ struct Fp8GemmArgs {
 
 template <int BN>
 struct Fp8Cfg {
-  static constexpr int A8 = 128 * 128;             // FP8 code tile
-  static constexpr int BB = BN * 64 * 2;           // one [BN x 64] bf16 tile
-  static constexpr int STAGE = A8 + 2 * BB;
-  static constexpr int ABF = 2 * 128 * 64 * 2;     // decoded A: two [128 x 64] f16 tiles
-  static constexpr int ST_RAW = (212 * 1024 - 2 * ABF - 1280) / STAGE;
-  static constexpr int STAGES = ST_RAW > 6 ? 6 : ST_RAW;
-  static constexpr int ABF_OFF = STAGES * STAGE;
-  static constexpr int BAR_OFF = ABF_OFF + 2 * ABF;
-  static constexpr int SMEM = 1024 + BAR_OFF + 256;
-  static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
+  static constexpr int A8 = 128 * 128;             // one FP8 code tile
+  static constexpr int BB = BN * 64 * 2;           // one [BN x 64] f16 token tile
+  static constexpr int TOK = 2 * BB;               // the tokens of one 128-wide K block
+  static constexpr int TS = 3;                     // token stages
+  static constexpr int CS_RAW = (226 * 1024 - TS * TOK - 1536) / A8;
+  static constexpr int CS = CS_RAW > 10 ? 10 : CS_RAW;   // code stages
+  static constexpr int TOK_OFF = CS * A8;
+  static constexpr int BAR_OFF = TOK_OFF + TS * TOK;
+  static constexpr int SMEM = 1024 + BAR_OFF + 512;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  // TMEM columns: decoded A buffers [0,64) [64,128) (f16 pairs), partials [128, 128 + NP BN)
+  static constexpr int NP = 3;   // partials: the MMAs run on while the fold stores a finished unit
+  static constexpr uint32_t TM_A = 0, TM_P = 128;
+  static constexpr int TMEM_COLS = (128 + NP * BN) <= 256 ? 256 : 512;
+  static constexpr int FOLD_WARPS = BN >= 32 ? 8 : 4;
 };
+constexpr int FP8_THREADS = 448;   // 4 decode, 8 fold, TMA, MMA warps
+constexpr int FP8_EPI_BLOCKS = 6;  // a unit's partial store, in K blocks of time (split choice)
 
 // Two E4M3 codes (low byte -> low half) to two f16 values.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes16) {
@@ -53,11 +64,8 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// warps 0-7 decode the codes (warpgroup h: k-half h of every row) and fold the
-// scaled partials (warpgroup h: column half h, or all columns by warps 0-3 when
-// BN < 32); warp 8 issues TMA, warp 9 the MMAs.
 template <int BN>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(FP8_THREADS, 1)
     tc_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        Fp8GemmArgs fa) {
   using C = Fp8Cfg<BN>;
@@ -66,30 +74,31 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar = sbase + C::BAR_OFF;
-  auto full_bar = [&](int s) { return bar + 8 * s; };
-  auto empty_bar = [&](int s) { return bar + 8 * (C::STAGES + s); };
-  const uint32_t conv_full = bar + 8 * (2 * C::STAGES);        // [2]
-  const uint32_t conv_free = conv_full + 16;                    // [2]
-  const uint32_t part_full = conv_free + 16;                    // [2]
-  const uint32_t part_free = part_full + 16;                    // [2]
-  const uint32_t fin = part_free + 16;
-  uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + 8 * (2 * C::STAGES) + 80);
-  volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+  const uint32_t code_full = bar, code_empty = bar + 8 * C::CS;          // [CS]
+  const uint32_t tok_full = bar + 16 * C::CS, tok_empty = tok_full + 8 * C::TS;   // [TS]
+  const uint32_t a_full = tok_empty + 8 * C::TS, a_free = a_full + 16;   // [2] decoded A in TMEM / consumed
+  const uint32_t part_full = a_free + 16, part_free = part_full + 8 * C::NP;   // [NP]
+  const uint32_t fin = part_free + 8 * C::NP;
+  uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + 480);
+  volatile int* abort_word = (volatile int*)(smem + C::BAR_OFF + 484);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int s = 0; s < C::CS; ++s) { mbar_init(code_full + 8 * s, 1); mbar_init(code_empty + 8 * s, 4); }
+    for (int s = 0; s < C::TS; ++s) { mbar_init(tok_full + 8 * s, 1); mbar_init(tok_empty + 8 * s, 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(conv_full + 8 * i, 256);
-      mbar_init(conv_free + 8 * i, 1);
+      mbar_init(a_full + 8 * i, 4);
+      mbar_init(a_free + 8 * i, 1);
+    }
+    for (int i = 0; i < C::NP; ++i) {
       mbar_init(part_full + 8 * i, 1);
-      mbar_init(part_free + 8 * i, BN >= 32 ? 256 : 128);
+      mbar_init(part_free + 8 * i, C::FOLD_WARPS);
     }
     mbar_init(fin, 1);
     *abort_word = 0;
     fence_mbar_init();
   }
-  if (warp == 8 && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
+  if (warp == 12 && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
   if (warp == 0) { tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -97,83 +106,108 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  if (warp == 8) {
-    // ---------------- TMA producer ----------------
+  if (warp == 12) {
+    // ---------------- TMA producer: the codes (the first CS ahead of the dependency wait: no
+    // earlier kernel writes the weights), and the tokens CS - TS K blocks behind them ----------------
     if (lane == 0) {
-      // the weight codes of the first STAGES k-blocks go out before the wait for
-      // the previous kernel (no earlier kernel of the stream writes them)
-      {
-        int it = 0;
-        for (int u = blockIdx.x; u < g.total_units && it < C::STAGES; u += gridDim.x) {
-          int mt, nt, b, s;
-          decode_unit(g, u, mt, nt, b, s);
-          const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
-          for (int kb = kb0; kb < kb1 && it < C::STAGES; ++kb, ++it) {
-            mbar_arrive_expect_tx(full_bar(it), C::STAGE);
-            tma_load_3d(sbase + it * C::STAGE, &tmA, full_bar(it), kb * 128, mt * 128, b);
+      constexpr int LAG = C::CS - C::TS;
+      // the (unit, K block) of the j-th K block of this CTA, walked twice: codes and tokens
+      struct Cursor {
+        int u, kb, kb1, mt, nt, b;
+        __device__ bool valid(const GemmArgs& g) const { return u < g.total_units; }
+        __device__ void enter(const GemmArgs& g) {
+          int s;
+          if (u < g.total_units) {
+            decode_unit(g, u, mt, nt, b, s);
+            kb = s * g.kb_per_split;
+            kb1 = min(g.k_blocks, kb + g.kb_per_split);
           }
         }
-      }
-      griddep_wait();
-      int it = 0;
+        __device__ void next(const GemmArgs& g) {
+          if (++kb >= kb1) {
+            u += gridDim.x;
+            enter(g);
+          }
+        }
+      };
+      Cursor cc{(int)blockIdx.x, 0, 0, 0, 0, 0}, tc{(int)blockIdx.x, 0, 0, 0, 0, 0};
+      cc.enter(g);
+      tc.enter(g);
+      int jc = 0, jt = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
-        int mt, nt, b, s;
-        decode_unit(g, u, mt, nt, b, s);
-        const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int st = it % C::STAGES;
-          const uint32_t dst = sbase + st * C::STAGE;
-          if (it >= C::STAGES) {
-            if (!mbar_wait(empty_bar(st), ((it / C::STAGES) & 1) ^ 1, abort_word, g.flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(full_bar(st), C::STAGE);
-            tma_load_3d(dst, &tmA, full_bar(st), kb * 128, mt * 128, b);
-          }
-          const int br = nt * BN;
-          if (g.b_rows_dim2) {
-            tma_load_3d(dst + C::A8, &tmB, full_bar(st), kb * 128, b, br);
-            tma_load_3d(dst + C::A8 + C::BB, &tmB, full_bar(st), kb * 128 + 64, b, br);
-          } else {
-            tma_load_3d(dst + C::A8, &tmB, full_bar(st), kb * 128, br, b);
-            tma_load_3d(dst + C::A8 + C::BB, &tmB, full_bar(st), kb * 128 + 64, br, b);
-          }
+      auto issue_codes = [&]() -> bool {
+        const int cs = jc % C::CS;
+        if (!mbar_wait(code_empty + 8 * cs, ((jc / C::CS) & 1) ^ 1, abort_word, g.flag)) return false;
+        mbar_arrive_expect_tx(code_full + 8 * cs, C::A8);
+        tma_load_3d(sbase + cs * C::A8, &tmA, code_full + 8 * cs, cc.kb * 128, cc.mt * 128, cc.b);
+        ++jc;
+        cc.next(g);
+        return true;
+      };
+      auto issue_tokens = [&]() -> bool {
+        const int ts = jt % C::TS;
+        if (!mbar_wait(tok_empty + 8 * ts, ((jt / C::TS) & 1) ^ 1, abort_word, g.flag)) return false;
+        const uint32_t dst = sbase + C::TOK_OFF + ts * C::TOK;
+        const int br = tc.nt * BN;
+        mbar_arrive_expect_tx(tok_full + 8 * ts, C::TOK);
+        if (g.b_rows_dim2) {
+          tma_load_3d(dst, &tmB, tok_full + 8 * ts, tc.kb * 128, tc.b, br);
+          tma_load_3d(dst + C::BB, &tmB, tok_full + 8 * ts, tc.kb * 128 + 64, tc.b, br);
+        } else {
+          tma_load_3d(dst, &tmB, tok_full + 8 * ts, tc.kb * 128, br, tc.b);
+          tma_load_3d(dst + C::BB, &tmB, tok_full + 8 * ts, tc.kb * 128 + 64, br, tc.b);
         }
+        ++jt;
+        tc.next(g);
+        return true;
+      };
+      while (ok && jc < C::CS && cc.valid(g)) ok = issue_codes();
+      griddep_wait();
+      while (ok && (cc.valid(g) || tc.valid(g))) {
+        if (tc.valid(g) && (jt + LAG <= jc || !cc.valid(g))) ok = issue_tokens();
+        else ok = issue_codes();
       }
-      const int first = it > C::STAGES ? it - C::STAGES : 0;
-      for (int j = first; j < it; ++j) {
+      for (int u = (jc > C::CS ? jc - C::CS : 0); u < jc; ++u) {   // loads still in flight land before exit
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(full_bar(j % C::STAGES), (j / C::STAGES) & 1))
+        while (!mbar_try_wait(code_full + 8 * (u % C::CS), (u / C::CS) & 1))
+          if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(g.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
+      }
+      for (int u = (jt > C::TS ? jt - C::TS : 0); u < jt; ++u) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(tok_full + 8 * (u % C::TS), (u / C::TS) & 1))
           if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(g.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ---------------- MMA issuer: one 128-wide K block into one TMEM partial ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, BN);
-      // descriptors built once; buffers and k-steps add their byte offset >> 4
-      const uint64_t da0 = sdesc_sw128(sbase + C::ABF_OFF), db0 = sdesc_sw128(sbase + C::A8);
-      int it = 0;
+      const uint64_t db0 = sdesc_sw128(sbase + C::TOK_OFF);
+      int j = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
         int mt, nt, b, s;
         decode_unit(g, u, mt, nt, b, s);
         const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int st = it % C::STAGES, cb = it & 1;
-          if (!mbar_wait(full_bar(st), (it / C::STAGES) & 1, abort_word, g.flag)) { ok = false; break; }
-          if (!mbar_wait(conv_full + 8 * cb, (it >> 1) & 1, abort_word, g.flag)) { ok = false; break; }
-          if (!mbar_wait(part_free + 8 * cb, ((it >> 1) & 1) ^ 1, abort_word, g.flag)) { ok = false; break; }
+        for (int kb = kb0; kb < kb1; ++kb, ++j) {
+          const int ts = j % C::TS, pb = j & 1, pp = j % C::NP;
+          if (!mbar_wait(a_full + 8 * pb, (j >> 1) & 1, abort_word, g.flag) ||
+              !mbar_wait(tok_full + 8 * ts, (j / C::TS) & 1, abort_word, g.flag) ||
+              !mbar_wait(part_free + 8 * pp, ((j / C::NP) & 1) ^ 1, abort_word, g.flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint64_t da = da0 + (uint64_t)(cb * (C::ABF / 16)), db = db0 + (uint64_t)(st * (C::STAGE / 16));
+          const uint64_t db = db0 + (uint64_t)(ts * (C::TOK / 16));
+          const uint32_t ta = tmem + C::TM_A + 64 * pb, td = tmem + C::TM_P + BN * pp;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              mma_bf16(tmem + cb * BN, da + (kk * 16384 + 32 * k) / 16, db + (kk * C::BB + 32 * k) / 16, idesc,
-                       (kk > 0 || k > 0) ? 1u : 0u);
-          mma_commit(part_full + 8 * cb);
-          mma_commit(conv_free + 8 * cb);
-          mma_commit(empty_bar(st));
+              mma_bf16_ts(td, ta + 32 * kk + 8 * k, db + (kk * C::BB + 32 * k) / 16, idesc, (kk > 0 || k > 0) ? 1u : 0u);
+          mma_commit(part_full + 8 * pp);
+          mma_commit(a_free + 8 * pb);
+          mma_commit(tok_empty + 8 * ts);
         }
       }
       mma_commit(fin);
@@ -181,80 +215,102 @@ __global__ void __launch_bounds__(320, 1)
       while (!mbar_try_wait(fin, 0))
         if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(g.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
     }
-  } else {
-    // ---------------- warps 0-7: decode codes, fold scaled partials, epilogue ----------------
-    griddep_wait();   // the output belongs to the stream's earlier kernels
-    constexpr int FSPLIT = BN >= 32 ? 2 : 1;   // warpgroups that fold
-    constexpr int NCOL = BN / FSPLIT;          // columns each folding thread owns
-    const int t = threadIdx.x;
-    const int r = t & 127;                     // A row of the tile = TMEM lane
-    const int half = t >> 7;                   // warpgroup: k-half to decode, column half to fold
-    const bool folds = half < FSPLIT;
-    const int col0 = half * NCOL;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    float acc[NCOL];
-    int it = 0;
+  } else if (warp < 4) {
+    // ---------------- decode: thread = weight row m of the tile = TMEM lane ----------------
+    const int m = threadIdx.x;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    int j = 0;
     bool ok = true;
-    // decode k-half `half` of row r of the A tile of iteration `j` (stage j % STAGES) into buffer j & 1
-    auto convert = [&](int j) -> bool {
-      const int st = j % C::STAGES, cb = j & 1;
-      if (!mbar_wait_warp(full_bar(st), (j / C::STAGES) & 1, abort_word, g.flag)) return false;
-      if (!mbar_wait_warp(conv_free + 8 * cb, ((j >> 1) & 1) ^ 1, abort_word, g.flag)) return false;
-      const uint8_t* arow = smem + st * C::STAGE + r * 128;
-      uint8_t* orow = smem + C::ABF_OFF + cb * C::ABF + half * 16384 + r * 128;
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {         // 16 codes = elements 16q .. 16q+15 of the row
-        const int q = 4 * half + qq;
-        const uint4 v = *reinterpret_cast<const uint4*>(arow + ((q ^ (r & 7)) << 4));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t outw[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          outw[2 * k] = e4m3x2_to_f16x2(w[k] & 0xFFFF);
-          outw[2 * k + 1] = e4m3x2_to_f16x2(w[k] >> 16);
-        }
-        const int c0 = 2 * qq;
-        *reinterpret_cast<uint4*>(orow + ((c0 ^ (r & 7)) << 4)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-        *reinterpret_cast<uint4*>(orow + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(outw[4], outw[5], outw[6], outw[7]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(conv_full + 8 * cb);
-      return true;
-    };
-    // the global iteration index of each work unit's first K block
-    int first_it = 0;
     for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
       int mt, nt, b, s;
       decode_unit(g, u, mt, nt, b, s);
       const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
-      const int nkb = kb1 - kb0;
-      first_it = it;
-#pragma unroll
-      for (int j = 0; j < NCOL; ++j) acc[j] = 0.f;
-      const float* sc = fa.scale + (long long)b * fa.scale_batch + (long long)mt * fa.scale_ld;
-      if (nkb > 0 && !convert(first_it)) { ok = false; break; }
-      for (int i = 0; i < nkb; ++i) {
-        const int j = first_it + i;
-        if (i + 1 < nkb && !convert(j + 1)) { ok = false; break; }
-        if (!folds) continue;
-        const int pb = j & 1;
-        if (!mbar_wait_warp(part_full + 8 * pb, (j >> 1) & 1, abort_word, g.flag)) { ok = false; break; }
+      for (int kb = kb0; kb < kb1; ++kb, ++j) {
+        const int cs = j % C::CS, pb = j & 1;
+        if (!mbar_wait_warp(code_full + 8 * cs, (j / C::CS) & 1, abort_word, g.flag) ||
+            !mbar_wait_warp(a_free + 8 * pb, ((j >> 1) & 1) ^ 1, abort_word, g.flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const float scl = sc[kb0 + i];
+        const uint8_t* arow = smem + cs * C::A8 + m * 128;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {   // 32 codes = elements 32 q4 .. 32 q4 + 31 -> 16 TMEM columns
+          uint32_t outw[16];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = 2 * q4 + h;
+            const uint4 v = *reinterpret_cast<const uint4*>(arow + ((q ^ (m & 7)) << 4));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              outw[8 * h + 2 * k] = e4m3x2_to_f16x2(w[k] & 0xFFFF);
+              outw[8 * h + 2 * k + 1] = e4m3x2_to_f16x2(w[k] >> 16);
+            }
+          }
+          tmem_st16(tmem + C::TM_A + 64 * pb + lane_base + 16 * q4, outw);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(code_empty + 8 * cs);   // the codes are in registers or TMEM
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(a_full + 8 * pb);
+      }
+    }
+  } else if (warp < 4 + C::FOLD_WARPS) {
+    // ---------------- fold: warps 4 .. 4 + FOLD_WARPS - 1, TMEM lane quarter warp % 4 ----------------
+    constexpr int FSPLIT = C::FOLD_WARPS / 4;  // column groups
+    constexpr int NCOL = BN / FSPLIT;          // columns each folding thread owns
+    const int w = warp - 4;
+    const int r = 32 * (warp & 3) + lane;      // A row of the tile = TMEM lane
+    const int col0 = (w >> 2) * NCOL;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    // The block scales of a unit, one unit ahead: lane l holds those of K blocks kb0 + l and
+    // kb0 + 32 + l, so a unit's first fold does not wait for a cold load behind the code stream.
+    auto load_scales = [&](int u, float& s0, float& s1) {
+      s0 = s1 = 0.f;
+      if (u >= g.total_units) return;
+      int mt, nt, b, s;
+      decode_unit(g, u, mt, nt, b, s);
+      const float* sc = fa.scale + (long long)b * fa.scale_batch + (long long)mt * fa.scale_ld;
+      const int kb0 = s * g.kb_per_split, nkb = min(g.k_blocks, kb0 + g.kb_per_split) - kb0;
+      if (lane < nkb) s0 = sc[kb0 + lane];
+      if (lane + 32 < nkb) s1 = sc[kb0 + 32 + lane];
+    };
+    float s0, s1;
+    load_scales(blockIdx.x, s0, s1);
+    griddep_wait();   // the output belongs to the stream's earlier kernels
+    float acc[NCOL];
+    int j = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
+      int mt, nt, b, s;
+      decode_unit(g, u, mt, nt, b, s);
+      const int kb0 = s * g.kb_per_split, kb1 = min(g.k_blocks, kb0 + g.kb_per_split);
+      const float c0 = s0, c1 = s1;
+      load_scales(u + gridDim.x, s0, s1);
+#pragma unroll
+      for (int c = 0; c < NCOL; ++c) acc[c] = 0.f;
+      const float* sc = fa.scale + (long long)b * fa.scale_batch + (long long)mt * fa.scale_ld;
+      for (int kb = kb0; kb < kb1; ++kb, ++j) {
+        const int pp = j % C::NP, i = kb - kb0;
+        const float scl = i < 32 ? __shfl_sync(0xffffffffu, c0, i) : i < 64 ? __shfl_sync(0xffffffffu, c1, i - 32) : sc[kb];
+        if (!mbar_wait_warp(part_full + 8 * pp, (j / C::NP) & 1, abort_word, g.flag)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < NCOL / 16; ++c) {
           uint32_t v[16];
-          tmem_ld16(tmem + pb * BN + col0 + lane_base + 16 * c, v);
+          tmem_ld16(tmem + C::TM_P + BN * pp + col0 + lane_base + 16 * c, v);
           tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 16; ++k) acc[16 * c + k] = fmaf(scl, __uint_as_float(v[k]), acc[16 * c + k]);
         }
         tc_fence_before();
-        mbar_arrive(part_free + 8 * pb);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(part_free + 8 * pp);
       }
       if (!ok) break;
-      it = first_it + nkb;
-      if (!folds) continue;
       const int m = mt * 128 + r;
 #pragma unroll
       for (int c = 0; c < NCOL / 16; ++c) {

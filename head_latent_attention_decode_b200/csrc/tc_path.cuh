@@ -158,7 +158,7 @@ static int launch_gemm_fp8_bn(const CUtensorMap& A, const CUtensorMap& B, const 
     attr_set[dev] = true;
   }
   const int grid = fa.g.total_units < num_sms ? fa.g.total_units : num_sms;
-  launch_pdl(tc_gemm_fp8_kernel<BN>, grid, 320, C::SMEM, s, A, B, fa);
+  launch_pdl(tc_gemm_fp8_kernel<BN>, grid, FP8_THREADS, C::SMEM, s, A, B, fa);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -187,15 +187,16 @@ static int launch_gemm_fp8(const CUtensorMap& A, const CUtensorMap& B, GemmArgs 
 }
 
 // Splits of the K loop for a persistent grid of num_sms CTAs: minimise the
-// work of the busiest CTA, ceil(m_tiles * s / num_sms) units of 1/s of K each
+// work of the busiest CTA, ceil(m_tiles * s / num_sms) units of 1/s of K each,
+// a unit costing its K blocks plus epi_blocks for storing its fp32 partial
 // (ties to fewer splits: fewer partial sums to add up afterwards).
-static int decode_splits_for(int m_tiles, int k_blocks, int num_sms) {
+static int decode_splits_for(int m_tiles, int k_blocks, int num_sms, int epi_blocks = 0) {
   int best = 1;
   double best_cost = 1e30;
   for (int s = 1; s <= 16 && s <= k_blocks; ++s) {
     const int per = (int)cdiv(k_blocks, s);
     const int real = (int)cdiv(k_blocks, per);          // the launcher drops empty splits
-    const double cost = (double)cdiv((long long)m_tiles * real, num_sms) * per;
+    const double cost = (double)cdiv((long long)m_tiles * real, num_sms) * (per + epi_blocks);
     if (cost < best_cost - 1e-9) { best_cost = cost; best = real; }
   }
   return best;
@@ -353,7 +354,7 @@ using namespace mla;
 using namespace mla::tc;
 
 struct TcDecodeWs {
-  size_t Yp, qn, q_nope, wo_part, bf16c, dq, total;
+  size_t Yp, qn, q_nope, wo_part, oy, bf16c, dq, total;
   int s1, s5;
   bool deq;   // FP8 weights beyond the FP8 GEMM's 128 tokens: dequantise each weight into dq, bf16 GEMMs
 };
@@ -367,14 +368,19 @@ static TcDecodeWs tc_decode_ws(const mla_handle* h, long long n) {
   const int sms = h->tc.num_sms > 0 ? h->tc.num_sms : 148;
   w.deq = h->tc.fp8 && n > 128;
   const int ku = h->tc.fp8 && !w.deq ? 128 : 64;   // K block of the GEMM kernel in use
-  w.s1 = decode_splits_for((int)cdiv(L.N1, 128), (int)cdiv(c.hidden, ku), sms);
-  w.s5 = decode_splits_for((int)cdiv(c.hidden, 128), (int)cdiv((long long)c.n_heads * c.v_dim, ku), sms);
+  // The FP8 kernel's fold warps store a finished unit themselves, behind the code stream: about
+  // six K blocks of time for a 128-token fp32 partial (the bf16 kernel's epilogue warps overlap it).
+  const int epi = h->tc.fp8 && !w.deq ? FP8_EPI_BLOCKS : 0;
+  w.s1 = decode_splits_for((int)cdiv(L.N1, 128), (int)cdiv(c.hidden, ku), sms, epi);
+  const long long ko = L.G ? (long long)L.G * L.ro : (long long)c.n_heads * c.v_dim;   // K of the last projection
+  w.s5 = decode_splits_for((int)cdiv(c.hidden, 128), (int)cdiv(ko, ku), sms, epi);
   size_t off = 0;
   auto put = [&](size_t b) { size_t o = off; off = align_up(off + b, 256); return o; };
   w.Yp = put((size_t)w.s1 * n * L.N1 * 4);
   w.qn = put((size_t)n * (c.q_lora_rank ? c.q_lora_rank : 8) * 2);
   w.q_nope = put((size_t)n * c.n_heads * c.qk_nope * 2);
   w.wo_part = put((size_t)w.s5 * n * c.hidden * 4);
+  if (L.G) w.oy = put((size_t)n * L.G * L.ro * 2);   // grouped output projection: the low-rank rows (bf16)
   if (w.deq) w.dq = put(tc_prefill_dequant_bytes(h));   // one dequantised weight at a time
   if (h->tc.fp8 && !w.deq) {   // f16 copy of the largest token operand of an FP8 GEMM
     long long e = c.hidden;
@@ -436,13 +442,24 @@ static inline int tc_init(mla_handle* h) {
   if (rq) st |= make_map2(&T.a_Wqb, b + L.Wqb, rq, L.Hq, rq, 128);
   st |= make_map(&T.a_Wuk, b + L.Wuk, dn, rkv, H, (long long)dn * 2, (long long)rkv * dn * 2, 128, 0);
   st |= make_map(&T.a_Wuv, b + L.Wuv, rkv, dv, H, (long long)rkv * 2, (long long)dv * rkv * 2, 128, 0);
-  st |= make_map2(&T.a_Wo, b + L.Wo, (long long)H * dv, D, (long long)H * dv, 128);
+  if (L.G) {
+    st |= make_map(&T.a_Woa, b + L.Woa, L.Kg, L.ro, L.G, (long long)L.Kg * 2, (long long)L.ro * L.Kg * 2, 128, 0);
+    st |= make_map2(&T.a_Wob, b + L.Wob, (long long)L.G * L.ro, D, (long long)L.G * L.ro, 128);
+  } else {
+    st |= make_map2(&T.a_Wo, b + L.Wo, (long long)H * dv, D, (long long)H * dv, 128);
+  }
   st |= make_map2(&T.b_W1, b + L.W1, D, L.N1, D, 256);
   st |= make_map2(&T.b_W1q, b + L.W1, D, L.Nq1, D, 256);
   st |= make_map2(&T.b_W1kv, b + L.W1 + (size_t)L.Nq1 * D * 2, D, L.R, D, 256);
   if (rq) st |= make_map2(&T.b_Wqb, b + L.Wqb, rq, L.Hq, rq, 256);
   st |= make_map2(&T.b_Wkvb, b + L.Wkvb, rkv, L.Hkv, rkv, 256);
-  st |= make_map2(&T.b_Wo, b + L.Wo, (long long)H * dv, D, (long long)H * dv, 256);
+  if (L.G) {
+    T.bn_oa = L.ro % 256 == 0 ? 256 : (L.ro % 128 == 0 ? 128 : 64);
+    st |= make_map(&T.b_Woa, b + L.Woa, L.Kg, L.ro, L.G, (long long)L.Kg * 2, (long long)L.ro * L.Kg * 2, T.bn_oa, 0);
+    st |= make_map2(&T.b_Wob, b + L.Wob, (long long)L.G * L.ro, D, (long long)L.G * L.ro, 256);
+  } else {
+    st |= make_map2(&T.b_Wo, b + L.Wo, (long long)H * dv, D, (long long)H * dv, 256);
+  }
   if (st != MLA_OK) return MLA_OK;   // stay on the CUDA-core path
   T.enabled = 1;
   return MLA_OK;
@@ -493,7 +510,7 @@ static inline int prefill_weight_map(const mla_handle* h, CUtensorMap* m, const 
   return make_map2(m, dq + (size_t)row0 * K * 2, K, rows, K, 256);
 }
 
-enum WSel { W_1, W_QB, W_UK, W_UV, W_O };
+enum WSel { W_1, W_QB, W_UK, W_UV, W_O, W_OA, W_OB };
 
 // Token operand of a decode GEMM: a bf16 3-D view {K, d1, d2} (strides in
 // elements) over `elems` contiguous elements, rows in dimension rows_dim2 + 1.
@@ -514,7 +531,8 @@ static int wgemm_body(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, 
 
 // Kernel-timer names of the decode weight GEMMs (mla_set_kernel_timer).
 static const char* wgemm_name(WSel w) {
-  return w == W_1 ? "gemm_w1" : w == W_QB ? "gemm_qb" : w == W_UK ? "gemm_uk" : w == W_UV ? "gemm_uv" : "gemm_o";
+  return w == W_1 ? "gemm_w1" : w == W_QB ? "gemm_qb" : w == W_UK ? "gemm_uk" : w == W_UV ? "gemm_uv"
+         : w == W_OA ? "gemm_oa" : w == W_OB ? "gemm_ob" : "gemm_o";
 }
 
 static int wgemm(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int bn, int splits, void* f16buf,
@@ -533,7 +551,8 @@ static int wgemm_body(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, 
   g.b_rows_dim2 = bv.rows_dim2;
   if (!T.fp8) {
     if ((st = make_map(&B, bv.p, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
-    const CUtensorMap* A = w == W_1 ? &T.a_W1 : w == W_QB ? &T.a_Wqb : w == W_UK ? &T.a_Wuk : w == W_UV ? &T.a_Wuv : &T.a_Wo;
+    const CUtensorMap* A = w == W_1 ? &T.a_W1 : w == W_QB ? &T.a_Wqb : w == W_UK ? &T.a_Wuk : w == W_UV ? &T.a_Wuv
+                           : w == W_OA ? &T.a_Woa : w == W_OB ? &T.a_Wob : &T.a_Wo;
     return launch_gemm(*A, B, g, bn, splits, T.num_sms, s);
   }
   if (dq) {
@@ -797,9 +816,22 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
   GemmArgs g4 = gemm_args(dv, n, rkv, H, EPI_BF16_T, head, (long long)H * dv, dv, flag);
   g4.b_rows_dim2 = 1;
   if ((st = wgemm(h, W_UV, vo, g4, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
-  // 3. out = head_out @ wo  (swap-AB, K split, then reduce to bf16)
-  GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
-  if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n), g5, bn, W.s5, f16buf, dq, s)) != MLA_OK) return st;
+  // 3. out = head_out @ wo  (swap-AB, K split, then reduce to bf16); or, grouped,
+  //    y[:, g] = head_out[:, group g] @ wo_a block g (batched over the groups:
+  //    A = Woa[g] [r_o, Kg], B = the group's head outputs), then out = y @ wo_b
+  const WeightLayout& L = h->L;
+  if (L.G) {
+    const BView vg{head, L.Kg, L.G, n, L.Kg, (long long)H * dv, (long long)n * H * dv, 1};
+    GemmArgs ga = gemm_args(L.ro, n, L.Kg, L.G, EPI_BF16_T, tw + W.oy, (long long)L.G * L.ro, L.ro, flag);
+    ga.b_rows_dim2 = 1;
+    if ((st = wgemm(h, W_OA, vg, ga, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
+    GemmArgs gb = gemm_args(D, n, L.G * L.ro, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
+    if ((st = wgemm(h, W_OB, bview2(tw + W.oy, (long long)L.G * L.ro, n), gb, bn, W.s5, f16buf, dq, s)) != MLA_OK)
+      return st;
+  } else {
+    GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
+    if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n), g5, bn, W.s5, f16buf, dq, s)) != MLA_OK) return st;
+  }
   const long long cnt = (long long)n * D;
   launch_pdl(splitk_reduce_bf16_kernel, (unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s,
              (const float*)(tw + W.wo_part), W.s5, cnt, (bf16*)out);
@@ -868,7 +900,7 @@ static inline int tc_v4_qkv(const mla_handle* h, const void* hidden, int S, cons
 static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, const float* cos, const float* sin,
                              void* out, void* head, void* kv_cache, int n_blocks, const int32_t* slot_mapping,
                              char* ws, size_t pY1, size_t pqn, size_t pQ, size_t pcn, size_t pkpe, size_t pKV,
-                             size_t pDQ, cudaStream_t s) {
+                             size_t pDQ, size_t pOY, cudaStream_t s) {
   const mla_config& c = h->cfg;
   const WeightLayout& L = h->L;
   const TcState& T = h->tc;
@@ -968,6 +1000,21 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
     prefill_attn_simt_kernel<bf16><<<dim3((unsigned)cdiv(S, PA_BQ), H), 128, smem, s>>>(pa);
     mla_timer_end("prefill_attn", s);
     mla_count_launch(1);
+  }
+  if (L.G) {
+    // grouped output projection: y[t][g r_o + j] = head[t, group g] @ wo_a block g
+    // (batched over the groups: A = the group's head outputs {Kg, S, G}, B = Woa),
+    // then out = y @ wo_b
+    CUtensorMap mg, my;
+    if ((st = make_map(&mg, head, L.Kg, S, L.G, (long long)H * dv * 2, (long long)L.Kg * 2, 128, 0)) != MLA_OK)
+      return st;
+    GemmArgs ga = gemm_args(S, L.ro, L.Kg, L.G, EPI_BF16_N, ws + pOY, (long long)L.G * L.ro, L.ro, flag);
+    ga.static_op = sop;
+    if ((st = launch_gemm(mg, T.b_Woa, ga, T.bn_oa, 1, T.num_sms, s)) != MLA_OK) return st;
+    if ((st = make_map2(&my, ws + pOY, (long long)L.G * L.ro, S, (long long)L.G * L.ro, 128)) != MLA_OK) return st;
+    GemmArgs gb = gemm_args(S, D, L.G * L.ro, 1, EPI_BF16_N, out, D, 0, flag);
+    gb.static_op = sop;
+    return launch_gemm(my, T.b_Wob, gb, 256, 1, T.num_sms, s);
   }
   CUtensorMap mh;
   if ((st = make_map2(&mh, head, (long long)H * dv, S, (long long)H * dv, 128)) != MLA_OK) return st;

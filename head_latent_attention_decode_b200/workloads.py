@@ -44,6 +44,8 @@ class MlaShape:
     weight_dtype: str         # "f32" | "bf16" | "fp8"
     norm_eps: float = 1e-6
     rope_theta: float = 10000.0
+    o_groups: int = 0         # DeepSeek-V4 grouped low-rank O: head groups (0 = one dense wo)
+    o_lora_rank: int = 0      # ... and each group's low rank
 
     @property
     def kv_row_dim(self) -> int:
@@ -152,7 +154,7 @@ def e4m3_encode(w_over_s: np.ndarray) -> np.ndarray:
 # weights
 # ----------------------------------------------------------------------------
 
-WEIGHT_NAMES = ("wq_a", "wq_b", "wkv_a", "wkv_b", "wo")
+WEIGHT_NAMES = ("wq_a", "wq_b", "wkv_a", "wkv_b", "wo", "wo_a", "wo_b")
 
 
 def weight_shapes(s: MlaShape) -> dict:
@@ -165,7 +167,13 @@ def weight_shapes(s: MlaShape) -> dict:
         d["wq_b"] = (s.hidden, s.q_out_dim)      # the full q_proj
     d["wkv_a"] = (s.hidden, s.kv_row_dim)
     d["wkv_b"] = (s.kv_lora_rank, s.n_heads * (s.qk_nope + s.v_dim))
-    d["wo"] = (s.n_heads * s.v_dim, s.hidden)
+    if s.o_lora_rank:
+        # grouped low-rank O: wo_a holds each group's [(H/G) d_v, r_o] block, the
+        # groups stacked along its input rows; wo_b [G r_o, D]
+        d["wo_a"] = (s.n_heads * s.v_dim, s.o_lora_rank)
+        d["wo_b"] = (s.o_groups * s.o_lora_rank, s.hidden)
+    else:
+        d["wo"] = (s.n_heads * s.v_dim, s.hidden)
     return d
 
 

@@ -90,6 +90,14 @@ typedef struct {
   int act_dtype;       /* mla_dtype: MLA_F32 or MLA_BF16 */
   int weight_dtype;    /* mla_dtype: must equal act_dtype, or MLA_FP8_E4M3_B128 */
   int row_layout;      /* mla_row_layout */
+  /* DeepSeek-V4 grouped low-rank output projection ("Struct MlaWeights",
+   * wo_a / wo_b / o_lora_rank: when o_lora_rank > 0 the decode and prefill
+   * paths use wo_a -> wo_b instead of wo; wo_a is sliced per o_group,
+   * block-diagonal). 0 / 0 = the dense wo. With o_lora_rank > 0: o_groups >= 1
+   * divides H; o_lora_rank and (H / o_groups) * d_v are multiples of 64; the
+   * weights are MLA_F32 or MLA_BF16. */
+  int o_groups;        /* G: consecutive head groups */
+  int o_lora_rank;     /* r_o: each group's low rank */
 } mla_config;
 
 /* Weights in [in, out] row-major form, device pointers, element type
@@ -99,7 +107,12 @@ typedef struct {
  *                                   q_proj [D, H*(d_n+d_r)]
  *   wkv_a [D, r_kv + d_r]           output order [latent | k_pe]
  *   wkv_b [r_kv, H*(d_n+d_v)]       per head [k_nope_h | v_h] columns
- *   wo    [H*d_v, D]
+ *   wo    [H*d_v, D]                (NULL when o_lora_rank > 0)
+ *   wo_a  [H*d_v, r_o]              o_lora_rank > 0 only: group g's block
+ *                                   [(H/G) d_v, r_o] in rows g (H/G) d_v ..;
+ *                                   it takes heads g (H/G) .. (g+1) (H/G) - 1
+ *   wo_b  [G*r_o, D]                o_lora_rank > 0 only: the groups' low-rank
+ *                                   outputs, concatenated in group order, -> D
  *   q_norm_w [r_q] fp32 (NULL when q_lora_rank == 0), kv_norm_w [r_kv] fp32
  *   *_scale: FP8 only, fp32 [ceil(in/128), ceil(out/128)], else NULL.
  *   attn_sink [H] fp32 or NULL: a per-head attention sink logit ("Struct
@@ -122,6 +135,8 @@ typedef struct {
   const float* wkv_b_scale;
   const float* wo_scale;
   const float* attn_sink;
+  const void* wo_a;
+  const void* wo_b;
 } mla_weights_desc;
 
 typedef struct mla_handle mla_handle;

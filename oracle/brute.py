@@ -49,6 +49,23 @@ def _softmax_row(s, sink=None):
     return [v / z for v in e]
 
 
+def _o_proj(cfg, W, head_out_t):
+    """One token's output projection from its head outputs [H][d_v]: wo, or the
+    grouped low-rank wo_a (per group of consecutive heads, its own block of
+    rows) then wo_b."""
+    flat = [v for h in head_out_t for v in h]
+    if not getattr(cfg, "o_lora_rank", 0):
+        return _vecmat(flat, _mat(W["wo"]))
+    G, ro = cfg.o_groups, cfg.o_lora_rank
+    kg = len(flat) // G
+    wo_a = _mat(W["wo_a"])
+    z = []
+    for g in range(G):
+        for j in range(ro):
+            z.append(sum(flat[g * kg + i] * wo_a[g * kg + i][j] for i in range(kg)))
+    return _vecmat(z, _mat(W["wo_b"]))
+
+
 def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens,
                 slot_mapping, layout=0, input_norm_w=None, inv_freq=None, attn_sink=None):
     """One whole decode step, loops only.
@@ -110,8 +127,7 @@ def decode_step(cfg, W, hidden, positions, cache_rows, block_table, context_lens
             o_t.append([sum(o_lat[cc] * wkv_b[cc][h * (dn + dv) + dn + d] for cc in range(rkv))
                         for d in range(dv)])
         head_out.append(o_t)
-    wo = _mat(W["wo"])
-    out = [_vecmat([v for h in range(H) for v in head_out[t][h]], wo) for t in range(len(hidden))]
+    out = [_o_proj(cfg, W, head_out[t]) for t in range(len(hidden))]
     return out, head_out, q_abs_all, q_pe_all, rows
 
 
@@ -153,8 +169,7 @@ def prefill(cfg, W, hidden, attn_sink=None):
             p = _softmax_row(s, None if attn_sink is None else float(attn_sink[h]))
             o_i.append([sum(p[j] * V[j][h][d] for j in range(i + 1)) for d in range(dv)])
         head_out.append(o_i)
-    wo = _mat(W["wo"])
-    out = [_vecmat([v for h in range(H) for v in head_out[i][h]], wo) for i in range(S)]
+    out = [_o_proj(cfg, W, head_out[i]) for i in range(S)]
     return out, head_out
 
 

@@ -314,6 +314,31 @@ def decode_qkv(cfg, W, hidden, cos, sin, kv_cache, slot_mapping, row_layout=LATE
     return q_abs, q_pe, cache
 
 
+def grouped_o_projection(head_out, wo_a, wo_b, o_groups):
+    """DeepSeek-V4 grouped low-rank output projection ("Struct MlaWeights",
+    wo_a / wo_b / o_lora_rank: wo_a -> wo_b replaces wo; wo_a is sliced per
+    o_group, block-diagonal). The heads split into o_groups consecutive groups;
+    group g's head outputs, flattened to [(H/G) d_v], go through its own block
+    wo_a[g] [(H/G) d_v, r_o] (rows g (H/G) d_v .. of wo_a); the G low-rank
+    vectors, concatenated in group order, go through wo_b [G r_o, D].
+    head_out [n, H, d_v] -> out [n, D]."""
+    n, H, dv = head_out.shape
+    G = o_groups
+    hg = H // G
+    wo_a = np.asarray(wo_a, np.float64)
+    z = [np.asarray(head_out[:, g * hg:(g + 1) * hg, :], np.float64).reshape(n, hg * dv)
+         @ wo_a[g * hg * dv:(g + 1) * hg * dv] for g in range(G)]
+    return np.concatenate(z, axis=1) @ np.asarray(wo_b, np.float64)
+
+
+def o_projection(cfg, W, head_out):
+    """out = concat_h(o[h]) @ wo, or the grouped low-rank wo_a -> wo_b when the
+    shape has o_lora_rank > 0 (grouped_o_projection)."""
+    if getattr(cfg, "o_lora_rank", 0):
+        return grouped_o_projection(head_out, W["wo_a"], W["wo_b"], cfg.o_groups)
+    return np.asarray(head_out, np.float64).reshape(head_out.shape[0], -1) @ np.asarray(W["wo"], np.float64)
+
+
 def decode_attn(cfg, W, q_abs, q_pe, kv_cache, block_table, context_lens,
                 row_layout=LATENT_FIRST, scale=None, attn_sink=None):
     """Absorbed attention over the latent cache, V extraction and o_proj.
@@ -339,7 +364,7 @@ def decode_attn(cfg, W, q_abs, q_pe, kv_cache, block_table, context_lens,
         p = softmax(s, axis=-1) if attn_sink is None else softmax_with_sink(s, attn_sink)
         o_lat = p @ c                                                      # [H, r_kv]
         head_out[t] = np.einsum("hc,hcd->hd", o_lat, w_uv)
-    out = head_out.reshape(n, -1) @ W["wo"]
+    out = o_projection(cfg, W, head_out)
     return out, head_out
 
 
@@ -363,7 +388,7 @@ def decode_attn_expanded(cfg, W, q_nope, q_pe, kv_cache, block_table, context_le
         s = (np.einsum("hp,hjp->hj", q_nope[t], k_nope) + q_pe[t] @ k_pe.T) * scale
         p = softmax(s, axis=-1)
         head_out[t] = np.einsum("hj,hjd->hd", p, v)
-    out = head_out.reshape(n, -1) @ W["wo"]
+    out = o_projection(cfg, W, head_out)
     return out, head_out
 
 
@@ -402,7 +427,7 @@ def prefill(cfg, W, hidden, cos, sin, rows=None, scale=None, row_layout=LATENT_F
              + q_pe[m] @ k_pe[:i + 1].T) * scale                       # [H, i+1]
         p = softmax(s, axis=-1) if attn_sink is None else softmax_with_sink(s, attn_sink)
         head_out[m] = np.einsum("hj,jhd->hd", p, v[:i + 1])
-    out = head_out.reshape(len(rows), -1) @ np.asarray(W["wo"], np.float64)
+    out = o_projection(cfg, W, head_out)
     return out, head_out, cache_row(c, k_pe, row_layout)
 
 
@@ -457,7 +482,7 @@ def weights_fp64(weights):
     """fp64 dict {wq_a?, wq_b, wkv_a, wkv_b, wo, q_norm_w?, kv_norm_w} from a
     workloads.Weights (dense values, or e4m3 codes + block scales)."""
     W = {}
-    for name in ("wq_a", "wq_b", "wkv_a", "wkv_b", "wo"):
+    for name in ("wq_a", "wq_b", "wkv_a", "wkv_b", "wo", "wo_a", "wo_b"):
         if name in weights.dense:
             W[name] = np.asarray(weights.dense[name], np.float64)
         elif name in weights.codes:

@@ -2,6 +2,7 @@
 every entry point include/mla.h declares, and rejects bad arguments before
 touching the device."""
 import ctypes
+import dataclasses
 import os
 import re
 
@@ -123,12 +124,13 @@ def test_calls_reject_null_handle_and_bad_sizes(lib):
     assert lib.mla_v4_qkv(None, P, -1, P, P, P, P, P, P, 1 << 20, None) == mla.MLA_ERR_INVALID_ARG
 
 
-def test_weights_descriptor_ends_with_the_sink():
-    """The C struct's field order: twelve weight / gamma / scale pointers, then
-    the optional attn_sink pointer (a zero-initialised descriptor has no sink)."""
+def test_weights_descriptor_field_order_matches_the_header():
+    """The C struct's field order: twelve weight / gamma / scale pointers, the
+    optional attn_sink pointer, then the grouped output projection's wo_a and
+    wo_b (a zero-initialised descriptor has neither)."""
     names = [f[0] for f in mla.mla_weights_desc._fields_]
-    assert names[-1] == "attn_sink" and len(names) == 13
-    assert ctypes.sizeof(mla.mla_weights_desc) == 13 * ctypes.sizeof(ctypes.c_void_p)
+    assert names[-3:] == ["attn_sink", "wo_a", "wo_b"] and len(names) == 15
+    assert ctypes.sizeof(mla.mla_weights_desc) == 15 * ctypes.sizeof(ctypes.c_void_p)
     hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "mla.h")).read()
     body = hdr[hdr.index("typedef struct {\n  const void* wq_a;"):hdr.index("} mla_weights_desc;")]
     fields = [ln.strip().rstrip(";").split()[-1].lstrip("*") for ln in body.splitlines()[1:] if ln.strip()]
@@ -150,3 +152,24 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         mla.mla_weights_bytes(mla.make_config(wl.TINY))
     with pytest.raises(ImportError):
         MlaLayer(wl.TINY, wl.make_weights(wl.TINY, 0), device="cpu")
+
+
+def test_config_field_order_matches_the_header():
+    names = [f[0] for f in mla.mla_config._fields_]
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "mla.h")).read()
+    body = hdr[hdr.index("typedef struct {\n  int hidden;"):hdr.index("} mla_config;")]
+    fields = [ln.split(";")[0].split()[-1] for ln in body.splitlines()[1:] if ln.strip().startswith(("int ", "float "))]
+    assert fields == names and names[-2:] == ["o_groups", "o_lora_rank"]
+
+
+def test_grouped_output_projection_config_checks(lib):
+    """o_lora_rank > 0 needs o_groups dividing H, 64-multiple sizes, and no FP8."""
+    base = wl.MlaShape(hidden=256, n_heads=4, q_lora_rank=64, kv_lora_rank=64, qk_nope=32, qk_rope=16,
+                       v_dim=32, block_size=16, act_dtype="f32", weight_dtype="f32")
+    ok = dataclasses.replace(base, o_groups=2, o_lora_rank=64)
+    assert mla.mla_weights_bytes(mla.make_config(ok)) > 0
+    for bad in (dataclasses.replace(base, o_groups=3, o_lora_rank=64),     # 3 does not divide 4 heads
+                dataclasses.replace(base, o_groups=0, o_lora_rank=64),
+                dataclasses.replace(base, o_groups=4, o_lora_rank=64),     # 32 inputs per group
+                dataclasses.replace(base, o_groups=2, o_lora_rank=48)):
+        assert mla.mla_weights_bytes(mla.make_config(bad)) == 0, bad

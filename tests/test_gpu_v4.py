@@ -120,3 +120,32 @@ def test_v4_qkv_needs_a_low_rank_query():
     with pytest.raises(mla.MlaError) as e:
         layer.v4_qkv(x, cos, sin, g)
     assert e.value.status == mla.MLA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
+# grouped low-rank output projection (wo_a -> wo_b)
+# ---------------------------------------------------------------------------
+
+def grouped(name, o_groups, o_lora_rank):
+    """The workload `name` with the grouped output projection in place of wo."""
+    w = wl.WORKLOADS[name]
+    return dataclasses.replace(w, shape=dataclasses.replace(w.shape, o_groups=o_groups, o_lora_rank=o_lora_rank))
+
+
+@pytest.mark.parametrize("name,groups,rank,batch,ctx", [
+    ("tiny_fp32", 2, 64, None, None),          # CUDA-core GEMVs
+    ("v2lite_bf16", 4, 128, 3, (100, 700)),    # tensor-core decode, few-head attention
+    ("v3_bf16", 16, 256, 5, (1, 900)),         # tensor-core decode, head-major attention
+])
+def test_grouped_output_projection_decode(name, groups, rank, batch, ctx):
+    case = DecodeCase(grouped(name, groups, rank), batch=batch, ctx=ctx).run()
+    check_case(case)
+
+
+@pytest.mark.parametrize("name,groups,rank,S", [
+    ("tiny_fp32", 2, 64, 40),
+    ("v3_prefill_bf16", 16, 256, 200),
+    ("v3_prefill_bf16", 8, 512, 129),
+])
+def test_grouped_output_projection_prefill(name, groups, rank, S):
+    run_prefill(grouped(name, groups, rank), S)

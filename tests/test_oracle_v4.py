@@ -238,3 +238,73 @@ def test_planted_missing_head_norm_is_caught(monkeypatch):
     assert mismatch() < 1e-12
     monkeypatch.setattr(ref, "head_rms", lambda q, eps: np.asarray(q, np.float64))
     assert mismatch() > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# grouped low-rank output projection (wo_a -> wo_b)
+# ---------------------------------------------------------------------------
+
+GROUPED = dataclasses.replace(wl.MlaShape(hidden=24, n_heads=4, q_lora_rank=12, kv_lora_rank=8, qk_nope=4,
+                                          qk_rope=4, v_dim=6, block_size=2, act_dtype="f32",
+                                          weight_dtype="f32"), o_groups=2, o_lora_rank=3)
+
+
+@pytest.mark.parametrize("shape", [GROUPED, dataclasses.replace(GROUPED, q_lora_rank=0, o_groups=4)])
+def test_decode_with_grouped_o_matches_brute_force(shape):
+    W, inp, cos, sin = _decode_case(shape, 31)
+    assert "wo" not in W and W["wo_a"].shape == (shape.n_heads * shape.v_dim, shape.o_lora_rank)
+    q_abs, q_pe, cache = ref.decode_qkv(shape, W, inp.hidden, cos, sin, inp.cache, inp.slot_mapping)
+    out, head_out = ref.decode_attn(shape, W, q_abs, q_pe, cache, inp.block_table, inp.context_lens)
+    b_out, b_head = brute.decode_step(shape, W, inp.hidden, inp.positions,
+                                      inp.cache.reshape(-1, shape.kv_row_dim).tolist(),
+                                      inp.block_table.tolist(), inp.context_lens, inp.slot_mapping)[:2]
+    np.testing.assert_allclose(head_out, np.array(b_head), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out, np.array(b_out), rtol=0, atol=1e-12)
+
+
+def test_prefill_with_grouped_o_matches_brute_force():
+    shape = GROUPED
+    W = _weights(shape, 32)
+    x = np.random.default_rng(32).standard_normal((5, shape.hidden))
+    cos, sin = ref.rope_cos_sin(np.arange(5), shape.qk_rope, shape.rope_theta)
+    out, head_out, _ = ref.prefill(shape, W, x, cos, sin)
+    b_out, b_head = brute.prefill(shape, W, x)
+    np.testing.assert_allclose(head_out, np.array(b_head), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out, np.array(b_out), rtol=0, atol=1e-12)
+
+
+def test_grouped_o_equals_its_block_diagonal_matrix():
+    """The grouped form is one block-diagonal [H d_v, G r_o] matrix (group g's
+    block on rows g (H/G) d_v.., columns g r_o..) followed by wo_b."""
+    rng = np.random.default_rng(33)
+    n, H, dv, G, ro, D = 3, 8, 5, 4, 3, 7
+    head = rng.standard_normal((n, H, dv))
+    wo_a, wo_b = rng.standard_normal((H * dv, ro)), rng.standard_normal((G * ro, D))
+    bd = np.zeros((H * dv, G * ro))
+    kg = H * dv // G
+    for g in range(G):
+        bd[g * kg:(g + 1) * kg, g * ro:(g + 1) * ro] = wo_a[g * kg:(g + 1) * kg]
+    want = head.reshape(n, -1) @ bd @ wo_b
+    np.testing.assert_allclose(ref.grouped_o_projection(head, wo_a, wo_b, G), want, rtol=1e-13, atol=1e-13)
+
+
+def test_one_group_is_the_low_rank_factorisation_of_wo():
+    """With one group the projection is the dense wo = wo_a @ wo_b."""
+    rng = np.random.default_rng(34)
+    head = rng.standard_normal((4, 6, 5))
+    wo_a, wo_b = rng.standard_normal((30, 2)), rng.standard_normal((2, 9))
+    np.testing.assert_allclose(ref.grouped_o_projection(head, wo_a, wo_b, 1),
+                               head.reshape(4, -1) @ (wo_a @ wo_b), rtol=1e-12, atol=1e-12)
+
+
+def test_planted_strided_head_groups_are_caught(monkeypatch):
+    """Groups of every G-th head instead of consecutive heads fail the pins."""
+    def strided(head_out, wo_a, wo_b, o_groups):
+        n, H, dv = head_out.shape
+        hg = H // o_groups
+        z = [np.asarray(head_out[:, g::o_groups, :], np.float64).reshape(n, hg * dv)
+             @ np.asarray(wo_a, np.float64)[g * hg * dv:(g + 1) * hg * dv] for g in range(o_groups)]
+        return np.concatenate(z, axis=1) @ np.asarray(wo_b, np.float64)
+    monkeypatch.setattr(ref, "grouped_o_projection", strided)
+    with pytest.raises(AssertionError):
+        test_decode_with_grouped_o_matches_brute_force(GROUPED)
