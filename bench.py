@@ -473,8 +473,20 @@ def cpu_oracle_sample(w: wl.Workload, budget_s: float = 12.0, max_reps: int = 10
                        f"{reps} oracle steps in {dt:.1f} s", seconds=dt)
 
 
-def run_ours(args, world, rank, local):
+def selected_workload(args) -> wl.Workload:
+    """The workload named on the command line, with the profiling-slice overrides
+    (--batch, --context) applied; the line's config then records the slice."""
+    import dataclasses
     w = wl.WORKLOADS[args.workload]
+    if args.batch and w.mode == "decode":
+        w = dataclasses.replace(w, batch=args.batch, name=f"{w.name}[batch={args.batch}]")
+    if args.context and w.mode == "decode":
+        w = dataclasses.replace(w, ctx_lo=args.context, ctx_hi=args.context, name=f"{w.name}[context={args.context}]")
+    return w
+
+
+def run_ours(args, world, rank, local):
+    w = selected_workload(args)
     peaks = {}
     pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk):
@@ -605,7 +617,7 @@ def run_reference(args, world, rank):
     bounded sample of the workload (set up once, outside the timing)."""
     if rank != 0:
         return None
-    w = wl.WORKLOADS[args.workload]
+    w = selected_workload(args)
     for _ in range(args.warmup):
         cpu_oracle_sample(w, budget_s=0.0, max_reps=1)
     vals, secs, cb = [], [], None
@@ -635,6 +647,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # profiling slices of a decode workload (fewer sequences, or one context for all); not bench lines
+    ap.add_argument("--batch", type=int, default=0, help="override the decode workload's sequence count")
+    ap.add_argument("--context", type=int, default=0, help="give every sequence this context length")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
