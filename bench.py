@@ -478,9 +478,9 @@ def selected_workload(args) -> wl.Workload:
     (--batch, --context) applied; the line's config then records the slice."""
     import dataclasses
     w = wl.WORKLOADS[args.workload]
-    if args.batch and w.mode == "decode":
+    if getattr(args, "batch", 0) and w.mode == "decode":
         w = dataclasses.replace(w, batch=args.batch, name=f"{w.name}[batch={args.batch}]")
-    if args.context and w.mode == "decode":
+    if getattr(args, "context", 0) and w.mode == "decode":
         w = dataclasses.replace(w, ctx_lo=args.context, ctx_hi=args.context, name=f"{w.name}[context={args.context}]")
     return w
 
