@@ -39,6 +39,7 @@ __device__ __forceinline__ float to_f32(uint8_t x) { return e4m3_to_f32(x); }
 template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
+template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -522,7 +522,7 @@ int mla_decode_attn(mla_handle* h, const void* q_abs, const void* q_pe, const vo
     const int r = tc_decode_attn(h, q_abs, q_pe, kv_cache, n_blocks, block_table, max_blocks_per_seq,
                                  context_lens, max_context_len, n, out, head, wsb, W.tc, s,
                                  (float*)(wsb + W.part_o), (float*)(wsb + W.part_ml), W.splits,
-                                 (bf16*)(wsb + W.o_lat), (int*)(wsb + W.nseg));
+                                 (bf16*)(wsb + W.o_lat), (int*)(wsb + W.nseg), head_out == nullptr);
     return r != MLA_OK ? r : cuda_status();
   }
   void* o_lat = wsb + W.o_lat;

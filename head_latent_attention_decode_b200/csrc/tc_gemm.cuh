@@ -44,6 +44,9 @@ struct GemmArgs {
   // weights): 1 = A, 2 = B, 0 = neither. Its first pipeline stages are loaded
   // before waiting for the previous kernel.
   int static_op;
+  // EPI_BF16_T and the q_nope part of EPI_QROPE_T write f16 instead of bf16
+  // (activations whose only reader is an FP8-weight GEMM, which takes f16 tokens)
+  int out_f16;
 };
 
 template <int BN>
@@ -73,11 +76,21 @@ __device__ __forceinline__ void gemm_store(const GemmArgs& g, int m, int n0, int
     }
     case EPI_BF16_T: {
       if (!m_ok) break;
-      bf16* o = (bf16*)g.out;
+      const long long base = (long long)b * g.bstride + m;
+      if (g.out_f16) {
+        __half* o = (__half*)g.out;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int n = n0 + j;
-        if (n < g.N) o[(long long)n * g.ldo + (long long)b * g.bstride + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        for (int j = 0; j < 16; ++j) {
+          const int n = n0 + j;
+          if (n < g.N) o[(long long)n * g.ldo + base] = __float2half_rn(__uint_as_float(r[j]));
+        }
+      } else {
+        bf16* o = (bf16*)g.out;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = n0 + j;
+          if (n < g.N) o[(long long)n * g.ldo + base] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        }
       }
       break;
     }
@@ -107,7 +120,9 @@ __device__ __forceinline__ void gemm_store(const GemmArgs& g, int m, int n0, int
         const int n = n0 + j;
         if (!m_ok || n >= g.N) continue;
         if (!rot) {
-          ((bf16*)g.out)[((long long)n * g.H + h) * g.dn + jj] = __float2bfloat16_rn(v);
+          const long long o = ((long long)n * g.H + h) * g.dn + jj;
+          if (g.out_f16) ((__half*)g.out)[o] = __float2half_rn(v);
+          else ((bf16*)g.out)[o] = __float2bfloat16_rn(v);
         } else {
           const float o = odd ? (partner * sn[j] + v * cs[j]) : (v * cs[j] - partner * sn[j]);
           ((bf16*)g.out2)[((long long)n * g.H + h) * g.dr + (jj - g.dn)] = __float2bfloat16_rn(o);

@@ -211,6 +211,7 @@ struct FrontFoldTcArgs {
   const float* q_norm_w; const float* kv_norm_w; float eps;
   const float* cos; const float* sin;
   bf16* qn; bf16* q_nope; bf16* q_pe;
+  int act_f16;   // qn and q_nope in f16 (their only reader is an FP8-weight GEMM)
   bf16* cache; long long n_rows; const int* slot; int layout;
   int* flag;
   int q_cols;   // columns of the q part per CTA: all r_q, or whole heads of d_n + d_r
@@ -269,13 +270,18 @@ __global__ void __launch_bounds__(512) frontfold_tc_kernel(FrontFoldTcArgs p) {
       float ss = 0.f;
       for (int i = threadIdx.x; i < p.rq; i += blockDim.x) ss += y[i] * y[i];
       const float r = rsqrtf(block_sum(ss, red) / (float)p.rq + p.eps);
-      for (int i = threadIdx.x; i < p.rq; i += blockDim.x)
-        p.qn[(long long)t * p.rq + i] = __float2bfloat16_rn(y[i] * r * p.q_norm_w[i]);
+      for (int i = threadIdx.x; i < p.rq; i += blockDim.x) {
+        const float v = y[i] * r * p.q_norm_w[i];
+        if (p.act_f16) ((__half*)p.qn)[(long long)t * p.rq + i] = __float2half_rn(v);
+        else p.qn[(long long)t * p.rq + i] = __float2bfloat16_rn(v);
+      }
     } else {
       const int hd = p.dn + p.dr, h0 = c0 / hd, nh = w / hd;
       for (int idx = threadIdx.x; idx < nh * p.dn; idx += blockDim.x) {
         const int h = idx / p.dn, j = idx % p.dn;
-        p.q_nope[((long long)t * p.H + h0 + h) * p.dn + j] = __float2bfloat16_rn(y[h * hd + j]);
+        const long long o = ((long long)t * p.H + h0 + h) * p.dn + j;
+        if (p.act_f16) ((__half*)p.q_nope)[o] = __float2half_rn(y[h * hd + j]);
+        else p.q_nope[o] = __float2bfloat16_rn(y[h * hd + j]);
       }
       for (int idx = threadIdx.x; idx < nh * half; idx += blockDim.x) {
         const int h = idx / half, i = idx % half;
@@ -518,14 +524,17 @@ struct BView {
   const void* p;
   long long K, d1, d2, s1, s2, elems;
   int rows_dim2;
+  int f16;   // the tokens are f16 already (an FP8-weight GEMM then reads them as they are)
 };
 
-static BView bview2(const void* p, long long K, long long rows) { return BView{p, K, rows, 1, K, K * rows, K * rows, 0}; }
+static BView bview2(const void* p, long long K, long long rows, int f16 = 0) {
+  return BView{p, K, rows, 1, K, K * rows, K * rows, 0, f16};
+}
 
 // Weight GEMM of the decode path: bf16 weights on tc_gemm_kernel, FP8 weights
-// on tc_gemm_fp8_kernel (tokens converted to f16 into `f16buf` first) with the
-// matrix's block scales, or, given `dq`, on tc_gemm_kernel after dequantising
-// the weight into it.
+// on tc_gemm_fp8_kernel (bf16 tokens converted to f16 into `f16buf` first,
+// f16 tokens read as they are) with the matrix's block scales, or, given `dq`,
+// on tc_gemm_kernel after dequantising the weight into it.
 static int wgemm_body(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, int bn, int splits, void* f16buf,
                       char* dq, cudaStream_t s);
 
@@ -586,12 +595,16 @@ static int wgemm_body(const mla_handle* h, WSel w, const BView& bv, GemmArgs g, 
     g.static_op = 0;
     return launch_gemm(A, B, g, bn, splits, T.num_sms, s);
   }
-  if ((((uintptr_t)bv.p) & 15) || (bv.elems % 8)) return MLA_ERR_UNSUPPORTED;
-  const long long n8 = bv.elems / 8;
-  const unsigned blocks = (unsigned)(cdiv(n8, 256) < 2048 ? cdiv(n8, 256) : 2048);
-  launch_pdl(cvt_bf16_f16_kernel, blocks, 256, 0, s, (const uint4*)bv.p, (uint4*)f16buf, n8);
-  mla_count_launch(1);
-  if ((st = make_map(&B, f16buf, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
+  const void* tok = bv.p;
+  if (!bv.f16) {
+    if ((((uintptr_t)bv.p) & 15) || (bv.elems % 8)) return MLA_ERR_UNSUPPORTED;
+    const long long n8 = bv.elems / 8;
+    const unsigned blocks = (unsigned)(cdiv(n8, 256) < 2048 ? cdiv(n8, 256) : 2048);
+    launch_pdl(cvt_bf16_f16_kernel, blocks, 256, 0, s, (const uint4*)bv.p, (uint4*)f16buf, n8);
+    mla_count_launch(1);
+    tok = f16buf;
+  }
+  if ((st = make_map(&B, tok, bv.K, bv.d1, bv.d2, bv.s1 * 2, bv.s2 * 2, bn, bv.rows_dim2)) != MLA_OK) return st;
   const WeightLayout& L = h->L;
   const mla_config& c = h->cfg;
   const char* base = h->base;
@@ -634,6 +647,8 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   // 1. Yp[split] = x @ W1 (swap-AB: A = W1 [N1, D], B = x [n, D])
   void* f16buf = tw + W.bf16c;
   char* dq = W.deq ? tw + W.dq : nullptr;
+  // with the FP8-weight GEMM, the activations only it reads are written in f16
+  const int af16 = h->tc.fp8 && !W.deq;
   GemmArgs g = gemm_args(L.N1, n, D, 1, EPI_F32_T, tw + W.Yp, L.N1, 0, flag);
   if ((st = wgemm(h, W_1, bview2(hidden, D, n), g, bn, W.s1, f16buf, dq, s)) != MLA_OK) return st;
   // 2. split sum, norms, RoPE, scatter (and, without q_lora, q_nope / q_pe)
@@ -643,7 +658,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   f.q_norm_w = rq ? (const float*)(h->base + L.gq) : nullptr;
   f.kv_norm_w = (const float*)(h->base + L.gkv); f.eps = c.norm_eps;
   f.cos = cos; f.sin = sin;
-  f.qn = (bf16*)(tw + W.qn); f.q_nope = (bf16*)(tw + W.q_nope); f.q_pe = (bf16*)q_pe;
+  f.qn = (bf16*)(tw + W.qn); f.q_nope = (bf16*)(tw + W.q_nope); f.q_pe = (bf16*)q_pe; f.act_f16 = af16;
   f.cache = (bf16*)kv_cache; f.n_rows = (long long)n_blocks * c.block_size; f.slot = slot_mapping;
   f.layout = c.row_layout; f.flag = flag;
   // the q part in slices: all of r_q (its RMSNorm spans it), or about a third
@@ -659,11 +674,11 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
   if (rq) {
 
     GemmArgs g2 = gemm_args(L.Hq, n, rq, 1, EPI_QROPE_T, tw + W.q_nope, 0, 0, flag);
-    g2.out2 = q_pe; g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr;
-    if ((st = wgemm(h, W_QB, bview2(tw + W.qn, rq, n), g2, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
+    g2.out2 = q_pe; g2.cos = cos; g2.sin = sin; g2.H = H; g2.dn = dn; g2.dr = dr; g2.out_f16 = af16;
+    if ((st = wgemm(h, W_QB, bview2(tw + W.qn, rq, n, af16), g2, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
   }
   // 4. q_abs[h] = q_nope[h] @ W_UK[h]  (batched over heads: A = Wuk[h] [r_kv, d_n], B = q_nope[:, h, :])
-  const BView vn{tw + W.q_nope, dn, H, n, dn, (long long)H * dn, (long long)n * H * dn, 1};
+  const BView vn{tw + W.q_nope, dn, H, n, dn, (long long)H * dn, (long long)n * H * dn, 1, af16};
   GemmArgs g3 = gemm_args(rkv, n, dn, H, EPI_BF16_T, q_abs, (long long)H * rkv, rkv, flag);
   g3.b_rows_dim2 = 1;
   return wgemm(h, W_UK, vn, g3, bn, 1, f16buf, dq, s);
@@ -674,7 +689,7 @@ static inline int tc_decode_qkv(const mla_handle* h, const void* hidden, int n, 
 static inline int tc_attention_core(const mla_handle* h, const void* q_abs, const void* q_pe, const void* kv_cache,
                                     int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
                                     int max_ctx, int n, float* part_o, float* part_ml, int splits, bf16* o_lat,
-                                    int* flag, int* nseg, cudaStream_t s) {
+                                    int* flag, int* nseg, cudaStream_t s, int olat_f16 = 0) {
   const mla_config& c = h->cfg;
   const TcState& T = h->tc;
   const int H = c.n_heads, dr = c.qk_rope, rkv = c.kv_lora_rank;
@@ -789,8 +804,12 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     mla_timer_end("attn", s);
     mla_count_launch(1);
   }
-  launch_pdl(attn_combine_kernel<bf16>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits, H,
-             rkv, o_lat, sink, ml_r, half_cols, (const int*)seg_counts);
+  if (olat_f16)   // its only reader is an FP8-weight GEMM
+    launch_pdl(attn_combine_kernel<__half>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits,
+               H, rkv, (__half*)o_lat, sink, ml_r, half_cols, (const int*)seg_counts);
+  else
+    launch_pdl(attn_combine_kernel<bf16>, dim3(n, H), 128, 0, s, (const float*)part_o, (const float*)part_ml, splits,
+               H, rkv, o_lat, sink, ml_r, half_cols, (const int*)seg_counts);
   mla_count_launch(1);
   return MLA_OK;
 }
@@ -799,38 +818,45 @@ static inline int tc_decode_attn(const mla_handle* h, const void* q_abs, const v
                                  int n_blocks, const int32_t* block_table, int mbps, const int32_t* ctx,
                                  int max_ctx, int n, void* out, void* head, char* ws, size_t tc_off,
                                  cudaStream_t s, float* part_o, float* part_ml, int splits, bf16* o_lat,
-                                 int* nseg) {
+                                 int* nseg, bool head_internal) {
   const mla_config& c = h->cfg;
   const TcDecodeWs W = tc_decode_ws(h, n);
   char* tw = ws + tc_off;
   int* flag = (int*)ws;
   const int H = c.n_heads, rkv = c.kv_lora_rank, dv = c.v_dim, D = c.hidden;
   const int bn = pick_bn(n);
+  // with the FP8-weight GEMM, o_lat, the head outputs (unless the caller asked for
+  // them) and the grouped low-rank rows are written in f16: only those GEMMs read them
+  const int af16 = h->tc.fp8 && !W.deq, hf16 = af16 && head_internal;
   int st = tc_attention_core(h, q_abs, q_pe, kv_cache, n_blocks, block_table, mbps, ctx, max_ctx, n, part_o,
-                             part_ml, splits, o_lat, flag, nseg, s);
+                             part_ml, splits, o_lat, flag, nseg, s, af16);
   if (st != MLA_OK) return st;
   // 2. head_out[h] = o_lat[h] @ W_UV[h]  (A = Wuv[h] [d_v, r_kv], B = o_lat[:, h, :])
   void* f16buf = tw + W.bf16c;
   char* dq = W.deq ? tw + W.dq : nullptr;
-  const BView vo{o_lat, rkv, H, n, rkv, (long long)H * rkv, (long long)n * H * rkv, 1};
+  const BView vo{o_lat, rkv, H, n, rkv, (long long)H * rkv, (long long)n * H * rkv, 1, af16};
   GemmArgs g4 = gemm_args(dv, n, rkv, H, EPI_BF16_T, head, (long long)H * dv, dv, flag);
   g4.b_rows_dim2 = 1;
+  g4.out_f16 = hf16;
   if ((st = wgemm(h, W_UV, vo, g4, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
   // 3. out = head_out @ wo  (swap-AB, K split, then reduce to bf16); or, grouped,
   //    y[:, g] = head_out[:, group g] @ wo_a block g (batched over the groups:
   //    A = Woa[g] [r_o, Kg], B = the group's head outputs), then out = y @ wo_b
   const WeightLayout& L = h->L;
   if (L.G) {
-    const BView vg{head, L.Kg, L.G, n, L.Kg, (long long)H * dv, (long long)n * H * dv, 1};
+    const BView vg{head, L.Kg, L.G, n, L.Kg, (long long)H * dv, (long long)n * H * dv, 1, hf16};
     GemmArgs ga = gemm_args(L.ro, n, L.Kg, L.G, EPI_BF16_T, tw + W.oy, (long long)L.G * L.ro, L.ro, flag);
     ga.b_rows_dim2 = 1;
+    ga.out_f16 = af16;
     if ((st = wgemm(h, W_OA, vg, ga, bn, 1, f16buf, dq, s)) != MLA_OK) return st;
     GemmArgs gb = gemm_args(D, n, L.G * L.ro, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
-    if ((st = wgemm(h, W_OB, bview2(tw + W.oy, (long long)L.G * L.ro, n), gb, bn, W.s5, f16buf, dq, s)) != MLA_OK)
+    if ((st = wgemm(h, W_OB, bview2(tw + W.oy, (long long)L.G * L.ro, n, af16), gb, bn, W.s5, f16buf, dq, s)) !=
+        MLA_OK)
       return st;
   } else {
     GemmArgs g5 = gemm_args(D, n, H * dv, 1, EPI_F32_T, tw + W.wo_part, D, 0, flag);
-    if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n), g5, bn, W.s5, f16buf, dq, s)) != MLA_OK) return st;
+    if ((st = wgemm(h, W_O, bview2(head, (long long)H * dv, n, hf16), g5, bn, W.s5, f16buf, dq, s)) != MLA_OK)
+      return st;
   }
   const long long cnt = (long long)n * D;
   launch_pdl(splitk_reduce_bf16_kernel, (unsigned)cdiv(cnt, 256) < 4096 ? (unsigned)cdiv(cnt, 256) : 4096, 256, 0, s,

@@ -120,6 +120,24 @@ def test_v3_fp8_full_sampled():
     check_case(case, seqs=[0, 64, 127])
 
 
+@pytest.mark.parametrize("batch", [3, 128])
+def test_v3_fp8_without_head_out(batch):
+    """Without a head_out buffer the FP8-weight step keeps its internal
+    activations (o_lat, the head outputs) in f16, the FP8 GEMM's token type;
+    `out` still matches the oracle, and the call that also returns head_out
+    (bf16) to within the same tolerance."""
+    case = DecodeCase(wl.WORKLOADS["v3_fp8"], batch=batch, ctx=(64, 700)).run()
+    out_with_head = to_np(case.out).copy()
+    out = case.layer.decode_attn(case.q_abs, case.q_pe, case.cache, case.table, case.ctx, case.max_ctx)
+    torch.cuda.synchronize()
+    seqs = [0, 1, 2] if batch == 3 else [0, 77, 127]
+    r = case.oracle(seqs)
+    tol = TOL[case.shape.act_dtype]
+    assert_close(to_np(out)[r["seqs"]], r["out"], tol, "out without head_out")
+    assert_close(to_np(out), out_with_head, tol, "out with and without head_out")
+    assert case.flag() == 0
+
+
 # ---------------------------------------------------------------------------
 # scatter exactness and device-side checks
 # ---------------------------------------------------------------------------

@@ -5,6 +5,8 @@ must not call cudaMalloc); its scratch is a fixed device array inside the
 library. Two calls in a row must both match mla_decode_qkv, since every call
 reuses the same array, and neither may take device memory. Collected last on
 purpose."""
+import gc
+
 import pytest
 import torch
 
@@ -29,6 +31,10 @@ def test_noalloc_front_fold_matches_regular_entry(name, batch, ctx):
     free_before, used_before = None, None
     for call in range(2):
         if call == 1:   # the first call has run: nothing more may be taken from the device
+            # tensors left unreachable by earlier tests are freed now, not by a
+            # collection in the middle of the measured call
+            gc.collect()
+            gc.disable()
             torch.cuda.synchronize()
             free_before, used_before = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
         q_abs, q_pe = outs[call]
@@ -36,6 +42,7 @@ def test_noalloc_front_fold_matches_regular_entry(name, batch, ctx):
                                    q_abs, q_pe)
         torch.cuda.synchronize()
         if call == 1:
+            gc.enable()
             assert torch.cuda.mem_get_info()[0] == free_before
             assert torch.cuda.memory_allocated() == used_before
         assert mla.mla_noalloc_read_device_flag() == 0
