@@ -13,7 +13,10 @@
 //   so the code stage is free again as soon as it is read;
 //   tcgen05 (kind::f16, A from TMEM, f16 x f16 -> fp32) multiplies that block
 //   alone into one of three TMEM partials;
-//   warps 4-11 add scale * partial to fp32 registers (two column halves);
+//   warps 4-11 add scale * partial to fp32 registers (two column halves) and,
+//   once a unit's K blocks are all folded, hand the tile to TMEM;
+//   warps 14-17 store it (the epilogue), so a store that waits behind the code
+//   stream holds up neither the fold nor the MMAs;
 //   warp 12 issues the TMA loads, warp 13 the MMAs.
 // So the scale multiplies each block's exact fp32 partial sum, the same value
 // as dequantising every weight in fp32 before the MAC, up to fp32 rounding.
@@ -43,13 +46,15 @@ struct Fp8Cfg {
   static constexpr int BAR_OFF = TOK_OFF + TS * TOK;
   static constexpr int SMEM = 1024 + BAR_OFF + 512;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-  // TMEM columns: decoded A buffers [0,64) [64,128) (f16 pairs), partials [128, 128 + NP BN)
-  static constexpr int NP = 3;   // partials: the MMAs run on while the fold stores a finished unit
-  static constexpr uint32_t TM_A = 0, TM_P = 128;
-  static constexpr int TMEM_COLS = (128 + NP * BN) <= 256 ? 256 : 512;
+  // TMEM columns: decoded A buffers [0,64) [64,128) (f16 pairs), partials [128, 128 + NP BN),
+  // the finished tile on its way out [128 + NP BN, 128 + (NP + 1) BN)
+  static constexpr int NP = BN >= 128 ? 2 : 3;
+  static constexpr uint32_t TM_A = 0, TM_P = 128, TM_OUT = 128 + NP * BN;
+  static constexpr int TMEM_COLS = (128 + (NP + 1) * BN) <= 256 ? 256 : 512;
+  static_assert(128 + (NP + 1) * BN <= 512, "TMEM columns");
   static constexpr int FOLD_WARPS = BN >= 32 ? 8 : 4;
 };
-constexpr int FP8_THREADS = 448;   // 4 decode, 8 fold, TMA, MMA warps
+constexpr int FP8_THREADS = 576;   // 4 decode, 8 fold, TMA, MMA, 4 epilogue warps
 constexpr int FP8_EPI_BLOCKS = 6;  // a unit's partial store, in K blocks of time (split choice)
 
 // Two E4M3 codes (low byte -> low half) to two f16 values.
@@ -79,6 +84,7 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
   const uint32_t a_full = tok_empty + 8 * C::TS, a_free = a_full + 16;   // [2] decoded A in TMEM / consumed
   const uint32_t part_full = a_free + 16, part_free = part_full + 8 * C::NP;   // [NP]
   const uint32_t fin = part_free + 8 * C::NP;
+  const uint32_t out_full = fin + 8, out_free = out_full + 8;                  // the finished tile in TMEM
   uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + 480);
   volatile int* abort_word = (volatile int*)(smem + C::BAR_OFF + 484);
 
@@ -95,6 +101,8 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
       mbar_init(part_free + 8 * i, C::FOLD_WARPS);
     }
     mbar_init(fin, 1);
+    mbar_init(out_full, C::FOLD_WARPS);
+    mbar_init(out_free, 4);
     *abort_word = 0;
     fence_mbar_init();
   }
@@ -263,7 +271,6 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
     constexpr int FSPLIT = C::FOLD_WARPS / 4;  // column groups
     constexpr int NCOL = BN / FSPLIT;          // columns each folding thread owns
     const int w = warp - 4;
-    const int r = 32 * (warp & 3) + lane;      // A row of the tile = TMEM lane
     const int col0 = (w >> 2) * NCOL;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     // The block scales of a unit, one unit ahead: lane l holds those of K blocks kb0 + l and
@@ -280,9 +287,8 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
     };
     float s0, s1;
     load_scales(blockIdx.x, s0, s1);
-    griddep_wait();   // the output belongs to the stream's earlier kernels
     float acc[NCOL];
-    int j = 0;
+    int j = 0, uo = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x) {
       int mt, nt, b, s;
@@ -311,14 +317,44 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
         if (lane == 0) mbar_arrive(part_free + 8 * pp);
       }
       if (!ok) break;
-      const int m = mt * 128 + r;
+      // hand the tile to the epilogue warps once they have read out the previous one
+      if (!mbar_wait_warp(out_free, (uo & 1) ^ 1, abort_word, g.flag)) break;
+      tc_fence_after();
 #pragma unroll
       for (int c = 0; c < NCOL / 16; ++c) {
         uint32_t outv[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) outv[k] = __float_as_uint(acc[16 * c + k]);
-        gemm_store(g, m, nt * BN + col0 + 16 * c, s, b, outv);
+        tmem_st16(tmem + C::TM_OUT + col0 + lane_base + 16 * c, outv);
       }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(out_full);
+      ++uo;
+    }
+  } else if (warp >= 14) {
+    // ---------------- epilogue: the finished tile, TMEM lane quarter warp % 4 -> global ----------------
+    griddep_wait();   // the output belongs to the stream's earlier kernels
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    int uo = 0;
+    for (int u = blockIdx.x; u < g.total_units; u += gridDim.x, ++uo) {
+      int mt, nt, b, s;
+      decode_unit(g, u, mt, nt, b, s);
+      if (!mbar_wait_warp(out_full, uo & 1, abort_word, g.flag)) break;
+      tc_fence_after();
+      const int m = mt * 128 + r;
+#pragma unroll 1
+      for (int c = 0; c < BN / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tmem + C::TM_OUT + lane_base + 16 * c, v);
+        tmem_ld_wait();
+        gemm_store(g, m, nt * BN + 16 * c, s, b, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(out_free);   // the fold may write the next tile
     }
   }
   tc_fence_before();
