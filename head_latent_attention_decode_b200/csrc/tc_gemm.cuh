@@ -49,6 +49,8 @@ struct GemmArgs {
   int out_f16;
 };
 
+constexpr int EPI_STG_BYTES = 2 * 8192;   // the transposed epilogue's staging (gemm_store_t16)
+
 template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
@@ -58,7 +60,8 @@ struct GemmCfg {
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
   static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;   // two accumulators
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = 1024 + BAR_OFF + 256;
+  static constexpr int STG_OFF = BAR_OFF + 256;   // the transposed epilogue's staging
+  static constexpr int SMEM = 1024 + STG_OFF + EPI_STG_BYTES;
 };
 
 __device__ __forceinline__ void gemm_store(const GemmArgs& g, int m, int n0, int split, int b, const uint32_t* r) {
@@ -206,6 +209,104 @@ __device__ __forceinline__ void gemm_store(const GemmArgs& g, int m, int n0, int
   }
 }
 
+// The transposed (swap-AB) epilogue modes through shared memory. The 128
+// epilogue threads (et = the tile row = TMEM lane) each hold their row's 16
+// columns n0 .. n0 + 15; those go into stg as [16 columns][128 rows] and leave
+// as 16-byte stores along m, so a warp's store instruction covers 512 contiguous
+// bytes instead of 32 scattered 2- or 4-byte values (under a saturated read
+// stream, such narrow stores took microseconds per tile). stg: two 8 KB
+// buffers, used by these 128 threads only; `chunk` counts the calls and picks
+// the buffer, and stg_bars[chunk & 1] (mbarriers of 4 arrivals, one per warp)
+// tell that all four warps have written it. Returns false if that wait gave up.
+__device__ __forceinline__ bool gemm_store_t16(const GemmArgs& g, int mt, int et, int n0, int split, int b,
+                                               uint32_t* v, uint8_t* stg_base, int chunk, uint32_t stg_bars,
+                                               volatile int* abort_word) {
+  const int m0 = mt * 128, m = m0 + et;
+  uint8_t* stg = stg_base + (chunk & 1) * 8192;
+  const int hd = g.dn + g.dr;
+  bool half_out = g.out_f16 != 0;   // 2-byte rows written as f16 (else bf16)
+  if (g.mode == EPI_QROPE_T) {
+    // rotate the q_pe rows (pairs of adjacent rows, i.e. lanes)
+    const int jj = m % hd;
+    const bool rot = m < g.M && jj >= g.dn;
+    const bool odd = (m & 1) != 0;
+    float cs[16], sn[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int n = n0 + j;
+      cs[j] = 1.f;
+      sn[j] = 0.f;
+      if (rot && n < g.N) {
+        const long long t = (long long)n * (g.dr >> 1) + ((jj - g.dn) >> 1);
+        cs[j] = g.cos[t];
+        sn[j] = g.sin[t];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float x = __uint_as_float(v[j]);
+      const float partner = __shfl_xor_sync(0xffffffffu, x, 1);   // all lanes take part
+      v[j] = __float_as_uint(odd ? (partner * sn[j] + x * cs[j]) : (x * cs[j] - partner * sn[j]));
+    }
+    half_out = half_out && !rot;   // q_pe stays bf16
+  }
+  // chunk - 1's writes are behind every thread, so chunk - 2's copy-out (same buffer) is done
+  if (g.mode == EPI_F32_T) {
+    float* st = (float*)stg;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) st[j * 128 + et] = __uint_as_float(v[j]);
+  } else {
+    __half* sh = (__half*)stg;
+    bf16* sb = (bf16*)stg;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (half_out) sh[j * 128 + et] = __float2half_rn(__uint_as_float(v[j]));
+      else sb[j * 128 + et] = __float2bfloat16_rn(__uint_as_float(v[j]));
+    }
+  }
+  __syncwarp();
+  const uint32_t sb_bar = stg_bars + 8 * (chunk & 1);
+  if ((et & 31) == 0) mbar_arrive(sb_bar);
+  if (!mbar_wait_warp(sb_bar, (chunk >> 1) & 1, abort_word, g.flag)) return false;
+  if (g.mode == EPI_F32_T) {
+#pragma unroll
+    for (int c = et; c < 512; c += 128) {   // [16 columns][32 groups of 4 rows]
+      const int j = c >> 5, mm = m0 + 4 * (c & 31), n = n0 + j;
+      if (n >= g.N || mm >= g.M) continue;
+      const float4 val = reinterpret_cast<const float4*>(stg)[c];
+      float* dst = (float*)g.out + ((long long)split * g.N + n) * g.ldo + mm;
+      if (mm + 4 <= g.M && (((uintptr_t)dst) & 15) == 0) {
+        *reinterpret_cast<float4*>(dst) = val;
+      } else {
+        const float e[4] = {val.x, val.y, val.z, val.w};
+        for (int k = 0; k < 4 && mm + k < g.M; ++k) dst[k] = e[k];
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = et; c < 256; c += 128) {   // [16 columns][16 groups of 8 rows]
+      const int j = c >> 4, mm = m0 + 8 * (c & 15), n = n0 + j;
+      if (n >= g.N || mm >= g.M) continue;
+      const uint4 val = reinterpret_cast<const uint4*>(stg)[c];
+      uint16_t* dst;
+      if (g.mode == EPI_BF16_T) {
+        dst = (uint16_t*)g.out + (long long)n * g.ldo + (long long)b * g.bstride + mm;
+      } else {   // QROPE: 8-row groups never straddle a head or its nope / rope boundary (d_n, d_r % 8 == 0)
+        const int h = mm / hd, jj = mm % hd;
+        dst = jj < g.dn ? (uint16_t*)g.out + ((long long)n * g.H + h) * g.dn + jj
+                        : (uint16_t*)g.out2 + ((long long)n * g.H + h) * g.dr + (jj - g.dn);
+      }
+      if (mm + 8 <= g.M && (((uintptr_t)dst) & 15) == 0) {
+        *reinterpret_cast<uint4*>(dst) = val;
+      } else {
+        const uint16_t* e = reinterpret_cast<const uint16_t*>(&val);
+        for (int k = 0; k < 8 && mm + k < g.M; ++k) dst[k] = e[k];
+      }
+    }
+  }
+  return true;
+}
+
 __device__ __forceinline__ void decode_unit(const GemmArgs& g, int u, int& mt, int& nt, int& b, int& s) {
   mt = u % g.m_tiles;
   u /= g.m_tiles;
@@ -232,12 +333,15 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t final_bar = bar + 8 * (2 * C::STAGES + 4);
   uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + 8 * (2 * C::STAGES + 5));
   volatile int* abort_word = (volatile int*)(tmem_slot + 1);
+  const uint32_t stg_bars = bar + 192;   // [2] the transposed epilogue's staging written (4 warps)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 128); }
     mbar_init(final_bar, 1);
+    mbar_init(stg_bars, 4);
+    mbar_init(stg_bars + 8, 4);
     *abort_word = 0;
     fence_mbar_init();
   }
@@ -344,7 +448,7 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ---------------- epilogue: warps 0..3 <-> TMEM lanes 32w..32w+31 ----------------
     griddep_wait();   // the output and the RoPE tables belong to the stream's earlier kernels
-    int tile = 0;
+    int tile = 0, chunk = 0;
     for (int u = blockIdx.x; u < g.total_units; u += gridDim.x, ++tile) {
       int mt, nt, b, s;
       decode_unit(g, u, mt, nt, b, s);
@@ -353,13 +457,21 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int m = mt * C::BM + warp * 32 + lane;
       const uint32_t row_addr = tmem + ((uint32_t)(warp * 32) << 16) + acc * BN;
+      // narrow tiles (few tokens) store directly: their staging round trip costs more than it saves
+      const bool staged = BN >= 64 && (g.mode == EPI_F32_T || g.mode == EPI_BF16_T || g.mode == EPI_QROPE_T);
+      bool ok = true;
 #pragma unroll 1
-      for (int c = 0; c < BN / 16; ++c) {
+      for (int c = 0; c < BN / 16 && ok; ++c) {
         uint32_t r[16];
         tmem_ld16(row_addr + c * 16, r);
         tmem_ld_wait();
-        gemm_store(g, m, nt * BN + c * 16, s, b, r);
+        if (staged)
+          ok = gemm_store_t16(g, mt, warp * 32 + lane, nt * BN + c * 16, s, b, r, smem + C::STG_OFF, chunk++,
+                              stg_bars, abort_word);
+        else
+          gemm_store(g, m, nt * BN + c * 16, s, b, r);
       }
+      if (!ok) break;
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }

@@ -40,11 +40,12 @@ struct Fp8Cfg {
   static constexpr int BB = BN * 64 * 2;           // one [BN x 64] f16 token tile
   static constexpr int TOK = 2 * BB;               // the tokens of one 128-wide K block
   static constexpr int TS = 3;                     // token stages
-  static constexpr int CS_RAW = (226 * 1024 - TS * TOK - 1536) / A8;
+  static constexpr int CS_RAW = (227 * 1024 - 1536 - EPI_STG_BYTES - TS * TOK) / A8;
   static constexpr int CS = CS_RAW > 10 ? 10 : CS_RAW;   // code stages
   static constexpr int TOK_OFF = CS * A8;
   static constexpr int BAR_OFF = TOK_OFF + TS * TOK;
-  static constexpr int SMEM = 1024 + BAR_OFF + 512;
+  static constexpr int STG_OFF = BAR_OFF + 512;   // the transposed epilogue's staging
+  static constexpr int SMEM = 1024 + STG_OFF + EPI_STG_BYTES;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   // TMEM columns: decoded A buffers [0,64) [64,128) (f16 pairs), partials [128, 128 + NP BN),
   // the finished tile on its way out [128 + NP BN, 128 + (NP + 1) BN)
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
   const uint32_t part_full = a_free + 16, part_free = part_full + 8 * C::NP;   // [NP]
   const uint32_t fin = part_free + 8 * C::NP;
   const uint32_t out_full = fin + 8, out_free = out_full + 8;                  // the finished tile in TMEM
+  const uint32_t stg_bars = out_free + 8;                                      // [2] epilogue staging written
   uint32_t* tmem_slot = (uint32_t*)(smem + C::BAR_OFF + 480);
   volatile int* abort_word = (volatile int*)(smem + C::BAR_OFF + 484);
 
@@ -103,6 +105,8 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
     mbar_init(fin, 1);
     mbar_init(out_full, C::FOLD_WARPS);
     mbar_init(out_free, 4);
+    mbar_init(stg_bars, 4);
+    mbar_init(stg_bars + 8, 4);
     *abort_word = 0;
     fence_mbar_init();
   }
@@ -338,19 +342,19 @@ __global__ void __launch_bounds__(FP8_THREADS, 1)
     griddep_wait();   // the output belongs to the stream's earlier kernels
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    int uo = 0;
-    for (int u = blockIdx.x; u < g.total_units; u += gridDim.x, ++uo) {
+    int uo = 0, chunk = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < g.total_units && ok; u += gridDim.x, ++uo) {
       int mt, nt, b, s;
       decode_unit(g, u, mt, nt, b, s);
       if (!mbar_wait_warp(out_full, uo & 1, abort_word, g.flag)) break;
       tc_fence_after();
-      const int m = mt * 128 + r;
 #pragma unroll 1
-      for (int c = 0; c < BN / 16; ++c) {
+      for (int c = 0; c < BN / 16 && ok; ++c) {
         uint32_t v[16];
         tmem_ld16(tmem + C::TM_OUT + lane_base + 16 * c, v);
         tmem_ld_wait();
-        gemm_store(g, m, nt * BN + 16 * c, s, b, v);
+        ok = gemm_store_t16(g, mt, r, nt * BN + 16 * c, s, b, v, smem + C::STG_OFF, chunk++, stg_bars, abort_word);
       }
       tc_fence_before();
       __syncwarp();
