@@ -175,8 +175,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   const uint32_t s_full = bar + 16 * ATT_NST;         // S_r(i) complete
   const uint32_t s_free = s_full + 8;                 // S read by the 8 softmax and 4 sender warps
   const uint32_t p_full_b = s_free + 8;               // [2] P(i) in shared memory (8 softmax warps)
-  const uint32_t x_full_b = p_full_b + 16;            // [2] peer partial landed
-  const uint32_t x_free_b = x_full_b + 16;            // [2] the peer's P.V has released its buffer
+  const uint32_t x_full_b = p_full_b + 16;            // [2 buffers][4 lane quarters] peer partial rows landed
+  const uint32_t x_free_b = x_full_b + 64;            // [2] the peer's P.V has released its buffer
   const uint32_t q_ready = x_free_b + 16;             // Q of the next segment in TMEM (8 softmax warps)
   const uint32_t o_done = q_ready + 8;                // each P.V
   const uint32_t o_seg = o_done + 8;                  // the last P.V of a segment
@@ -203,7 +203,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     mbar_init(s_free, 12);
     for (int i = 0; i < 2; ++i) {
       mbar_init(p_full_b + 8 * i, 8);
-      mbar_init(x_full_b + 8 * i, 1);
+      for (int k = 0; k < 4; ++k) mbar_init(x_full_b + 8 * (4 * i + k), 1);
       mbar_init(x_free_b + 8 * i, 1);
     }
     mbar_init(q_ready, 8);
@@ -342,12 +342,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
     }
   } else if (warp >= 10) {
-    // ---------------- senders: S_r(i) -> staging -> one bulk copy into the peer's X ----------------
-    const int h = 32 * (warp & 3) + lane;                 // TMEM lane quarter of this warp
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const bool issuer = (warp == 10 && lane == 0);
+    // ---------------- senders: S_r(i) -> staging -> per warp, one bulk copy of its 32 rows into the
+    // peer's X, landing on that quarter's barrier (the peer's softmax warps of the quarter wait for it alone)
+    const int qs = warp & 3;                              // TMEM lane quarter of this warp
+    const int h = 32 * qs + lane;
+    const uint32_t lane_base = (uint32_t)(qs * 32) << 16;
     const uint32_t peer_x = mapa_shared(x_s, peer), peer_x_full = mapa_shared(x_full_b, peer);
-    const uint32_t stg_s = sbase + SM::STG_OFF;
+    const uint32_t stg_s = sbase + SM::STG_OFF + 4096 * qs;   // this warp's rows, 4 KB
     uint4* stg_row = (uint4*)(smem + SM::STG_OFF + h * 128);
     for (int i = 0; i < N; ++i) {
       if (!mbar_wait_warp(s_full, i & 1, abort_word, a.flag)) break;
@@ -360,8 +361,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
-      if (issuer) bulk_wait_read_all();                  // the previous copy has left the staging buffer
-      named_bar_sync(2, 128);
+      if (lane == 0) bulk_wait_read_all();               // this warp's previous copy has left its rows
+      __syncwarp();
       // the partial goes out in f16 (half the distributed-shared-memory bytes of fp32; the
       // partial scores stay far inside f16's range and its 11-bit significand costs the
       // scores ~1e-3 relative, well inside the output tolerance)
@@ -376,17 +377,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         stg_row[k ^ (h & 7)] = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
-      named_bar_sync(2, 128);
-      if (issuer) {
+      __syncwarp();
+      if (lane == 0) {
         // the peer's P.V(i - 2) has released the buffer we send into
         const int xb = i & 1;
         if (mbar_wait_cluster(x_free_b + 8 * xb, ((i >> 1) & 1) ^ 1, abort_word, a.flag)) {
-          bulk_copy_to_peer(peer_x + xb * 16384, stg_s, 16384, peer_x_full + 8 * xb);
+          bulk_copy_to_peer(peer_x + xb * 16384 + 4096 * qs, stg_s, 4096, peer_x_full + 8 * (4 * xb + qs));
           bulk_commit_group();
         }
       }
     }
-    if (issuer) bulk_wait_read_all();
+    if (lane == 0) bulk_wait_read_all();
   } else {
     // ---------------- softmax: head h <-> TMEM lane h, columns [32 g, 32 g + 32) of each tile ----------------
     const int q = warp & 3, g = warp >> 2;
@@ -441,7 +442,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         blk_next = tile_block(wn);
       }
       const int valid = (blk >= 0 && blk < a.n_blocks) ? min(64, seq_len - 64 * lt) : 0;
-      if (threadIdx.x == 0) mbar_arrive_expect_tx(x_full_b + 8 * xb, 16384);
+      if (g == 0 && lane == 0) mbar_arrive_expect_tx(x_full_b + 8 * (4 * xb + q), 4096);   // this quarter's rows
       if (!mbar_wait_warp(s_full, i & 1, abort_word, a.flag)) { ok = false; break; }
       tc_fence_after();
       float v[32];
@@ -452,7 +453,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);   // the next S may overwrite the buffer
-      if (!mbar_wait_warp(x_full_b + 8 * xb, (i >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
+      if (!mbar_wait_warp(x_full_b + 8 * (4 * xb + q), (i >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       // row h, chunks 4 g .. 4 g + 3 of the peer's partial; P(i) later goes to exactly these bytes
       uint4* xrow = (uint4*)(smem + SM::X_OFF + xb * 16384 + h * 128);
 #pragma unroll
