@@ -13,7 +13,8 @@
 // are padded with zeros). CTA r owns latent columns [256 r, 256 r + 256) of
 // every tile and the 64 rotary columns of the tiles with odd-even index r:
 //   S_r = [q_abs | q_pe]_r . tile_r^T      (tcgen05, M 128 x N 64, K 256 or 320;
-//                                          Q lives in TMEM)
+//                                          the latent part of Q lives in TMEM,
+//                                          q_pe in shared memory; two S buffers)
 //   S   = S_r + S_peer                     (the partials swap through DSMEM in
 //                                          f16, into two alternating buffers)
 //   online softmax, two threads per head (each half of the tile's 64 columns;
@@ -25,11 +26,14 @@
 //                                          M 128 x N 256, K 64; V = the same
 //                                          shared-memory tile read MN-major)
 // Every cache byte is read from HBM once and O (128 x 512 fp32) is split over
-// the two CTAs' TMEM. A tile's ring stage is held from its load until its
-// P.V, so the shared memory left over by the exchange buffers goes to a
-// 4-deep ring; the S buffer is released as soon as the softmax and the sender
-// have read it. Warps 0-7 run the softmax (warp w: TMEM lane quarter w % 4,
-// column half w / 4), warp 8 issues TMA, warp 9 the MMAs, and warps 10-13 send
+// the two CTAs' TMEM. A tile's latent stage is held from its load until its
+// P.V, its rotary block (every other tile) only until its S, so the latent
+// blocks have a 4-deep ring and the rotary blocks 2 slots of their own. S
+// alternates between two TMEM buffers, so S(i + 1) runs, and its partial
+// crosses to the peer, while the softmax still works on S(i). Warps 0-7 run
+// the softmax (warp w: TMEM lane quarter w % 4, column half w / 4), warp 8
+// issues TMA, warp 9 the score MMAs and warp 14 the P.V MMAs (one thread each,
+// so a P.V never waits behind the issue of a later S), and warps 10-13 send
 // each tile's partial scores to the peer as soon as S lands.
 #pragma once
 
@@ -61,21 +65,25 @@ struct TcAttnArgs {
   int* nseg;
 };
 
-constexpr int ATT_NST = 4;                      // tile ring depth
-constexpr int ATT_THREADS = 448;                // 8 softmax, 1 TMA, 1 MMA, 4 sender warps
+constexpr int ATT_NST = 4;                      // latent ring depth
+constexpr int ATT_NRP = 2;                      // rotary slots (the tiles of this CTA's parity)
+constexpr int ATT_THREADS = 480;                // 8 softmax, 1 TMA, 1 S-MMA, 4 sender, 1 P.V-MMA warps
 constexpr int ATT_MAX_SEQ = 256;                // sequences per call (the prefix table in shared memory)
 struct AttnSmem {
-  static constexpr int STAGE = 5 * 8192;        // 4 latent + 1 rope slot of [64 rows x 64 cols] bf16
+  static constexpr int STAGE = 4 * 8192;        // the 4 latent k-blocks of [64 rows x 64 cols] bf16
   static constexpr int TILE_OFF = 0;
-  static constexpr int X_OFF = ATT_NST * STAGE;   // 2 x [128 x 64] f16 peer partial S, then P (bf16) over it
+  static constexpr int ROPE_OFF = ATT_NST * STAGE;          // ATT_NRP x [64 x 64] bf16 rotary blocks
+  static constexpr int QPE_OFF = ROPE_OFF + ATT_NRP * 8192;   // [128 x 64] bf16 q_pe (MMA operand layout)
+  static constexpr int X_OFF = QPE_OFF + 16384;   // 2 x [128 x 64] f16 peer partial S, then P (bf16) over it
   static constexpr int STG_OFF = X_OFF + 32768;   // [128 x 64] f16, our partial on its way out
   static constexpr int RED_OFF = STG_OFF + 16384; // [2 tiles][2 halves][128] fp32 half-row maxima, then [128] l
   static constexpr int PREF_OFF = RED_OFF + 2 * 2 * 128 * 4 + 128 * 4;   // [ATT_MAX_SEQ + 1] tile prefix sums
   static constexpr int BAR_OFF = PREF_OFF + (ATT_MAX_SEQ + 4) * 4;
   static constexpr int SIZE = 1024 + BAR_OFF + 512;
+  static_assert(SIZE <= 227 * 1024, "shared memory per CTA");
 };
-// TMEM columns: Q latent [0,128) and q_pe [128,160) (bf16 pairs), S [192,256), O [256,512)
-constexpr uint32_t ATT_TM_Q = 0, ATT_TM_QPE = 128, ATT_TM_S = 192, ATT_TM_O = 256;
+// TMEM columns: Q latent [0,128) (bf16 pairs), S buffers [128,192) [192,256), O [256,512)
+constexpr uint32_t ATT_TM_Q = 0, ATT_TM_S = 128, ATT_TM_O = 256;
 
 // Walks a cluster's slice of the batch's tile list: sequence b, its tile lt.
 struct TileWalk {
@@ -172,9 +180,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   // barriers (8 B each)
   const uint32_t full_b = bar;                        // [ATT_NST] tile landed
   const uint32_t empty_b = bar + 8 * ATT_NST;         // [ATT_NST] tile consumed by P.V
-  const uint32_t s_full = bar + 16 * ATT_NST;         // S_r(i) complete
-  const uint32_t s_free = s_full + 8;                 // S read by the 8 softmax and 4 sender warps
-  const uint32_t p_full_b = s_free + 8;               // [2] P(i) in shared memory (8 softmax warps)
+  const uint32_t s_full = bar + 16 * ATT_NST;         // [2] S_r(i) complete, in buffer i & 1
+  const uint32_t s_free = s_full + 16;                // [2] S read by the 8 softmax and 4 sender warps
+  const uint32_t p_full_b = s_free + 16;              // [2] P(i) in shared memory (8 softmax warps)
   const uint32_t x_full_b = p_full_b + 16;            // [2 buffers][4 lane quarters] peer partial rows landed
   const uint32_t x_free_b = x_full_b + 64;            // [2] the peer's P.V has released its buffer
   const uint32_t q_ready = x_free_b + 16;             // Q of the next segment in TMEM (8 softmax warps)
@@ -184,8 +192,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   const uint32_t fin = o_free + 8;
   const uint32_t xch_b = fin + 8;                     // [4 quarters][2] the two halves' maxima posted
   const uint32_t l_done = xch_b + 64;                 // [4] the second half's row sums posted
-  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 320);
-  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 324);
+  const uint32_t rope_empty = l_done + 32;            // [ATT_NRP] rotary block consumed by S
+  uint32_t* tmem_slot = (uint32_t*)(smem + SM::BAR_OFF + 448);
+  volatile int* abort_word = (volatile int*)(smem + SM::BAR_OFF + 452);
 
   const uint32_t r = cluster_ctarank(), peer = r ^ 1u;
   const int c = blockIdx.x >> 1;
@@ -199,8 +208,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ATT_NST; ++i) { mbar_init(full_b + 8 * i, 1); mbar_init(empty_b + 8 * i, 1); }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 12);
+    for (int i = 0; i < 2; ++i) { mbar_init(s_full + 8 * i, 1); mbar_init(s_free + 8 * i, 12); }
+    for (int i = 0; i < ATT_NRP; ++i) mbar_init(rope_empty + 8 * i, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(p_full_b + 8 * i, 8);
       for (int k = 0; k < 4; ++k) mbar_init(x_full_b + 8 * (4 * i + k), 1);
@@ -210,7 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     mbar_init(o_done, 1);
     mbar_init(o_seg, 1);
     mbar_init(o_free, 8);
-    mbar_init(fin, 1);
+    mbar_init(fin, 2);   // both issuing threads' last commits
     for (int i = 0; i < 8; ++i) mbar_init(xch_b + 8 * i, 2);
     for (int i = 0; i < 4; ++i) mbar_init(l_done + 8 * i, 1);
     *abort_word = 0;
@@ -241,18 +250,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       }
       const int blk = __shfl_sync(0xffffffffu, blkv, i & 31);
       const int st = i % ATT_NST;
+      const bool rope = (i & 1) == (int)r;
+      const int ri = (i >> 1) % ATT_NRP;
       if (!mbar_wait_warp(empty_b + 8 * st, ((i / ATT_NST) & 1) ^ 1, abort_word, a.flag)) break;
+      if (rope && !mbar_wait_warp(rope_empty + 8 * ri, (((i >> 1) / ATT_NRP) & 1) ^ 1, abort_word, a.flag)) break;
       if (lane == 0) {
         const int j0 = 64 * w.lt;
         long long row = -64;
         if (blk >= 0 && blk < a.n_blocks) row = (long long)blk * a.bs + (j0 % a.bs);
         else if (r == 0) set_flag(a.flag, MLA_FLAG_BAD_BLOCK);
-        const bool rope = (i & 1) == (int)r;
         mbar_arrive_expect_tx(full_b + 8 * st, rope ? 5 * 8192 : 4 * 8192);
         const uint32_t dst = tile_s + st * SM::STAGE;
         // the 4 latent k-blocks of the 64 rows in one box: [8 row octets][4 k-blocks][8 rows][128 B]
         tma_load_4d(dst, &tm_lat, full_b + 8 * st, 0, 0, a.lat_col0 / 64 + 4 * (int)r, (int)(row / 8));
-        if (rope) tma_load_3d(dst + 4 * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
+        if (rope) tma_load_3d(sbase + SM::ROPE_OFF + ri * 8192, &tm_cache, full_b + 8 * st, a.rope_col0, (int)row, 0);
       }
     }
     // drain the loads still in flight
@@ -264,84 +275,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       }
     }
   } else if (warp == 9) {
-    // ---------------- MMA issuer: P.V of the oldest tile first, else the next S ----------------
+    // ---------------- S issuer: S(t) into buffer t & 1 once its tile has landed ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64);
-      constexpr uint32_t idesc_o = idesc_bf16(128, 256, 1);
       // descriptors built once; stages and k-steps add their byte offset >> 4
-      const uint64_t d_t = sdesc_sw128_sbo(tile_s, 4096), d_rope = sdesc_sw128(tile_s + 4 * 8192);
-      const uint64_t d_v = sdesc_sw128_mn_sbo(tile_s, 1024, 4096), d_p = sdesc_sw128(x_s);
-      TileWalk ws{pref, a.n, 0, 0}, wo{pref, a.n, 0, 0};
+      const uint64_t d_t = sdesc_sw128_sbo(tile_s, 4096), d_rope = sdesc_sw128(sbase + SM::ROPE_OFF);
+      const uint64_t d_qpe = sdesc_sw128(sbase + SM::QPE_OFF);
+      TileWalk ws{pref, a.n, 0, 0};
       ws.start(g0);
-      wo.start(g0);
-      int next_s = 0, next_o = 0, ks = 0, ko = 0;
-      bool ok = true;
-      uint64_t t_last = global_timer_ns();
-      while (ok && next_o < N) {
-        bool did = false;
-        if (next_o < next_s) {
-          const int u = next_o, st = u % ATT_NST, xb = u & 1;
-          const bool first = (u == 0 || wo.lt == 0), last = (u == N - 1 || wo.seg_last());
-          if (mbar_test(p_full_b + 8 * xb, (u >> 1) & 1) && (!first || ko == 0 || mbar_test(o_free, (ko - 1) & 1))) {
-            tc_fence_after();
-            const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
-            const uint64_t dp = d_p + (uint64_t)(xb * (16384 / 16));
+      int ks = 0;
+      for (int t = 0; t < N; ++t, ws.next()) {
+        const int st = t % ATT_NST;
+        const bool first = (t == 0 || ws.lt == 0), last = (t == N - 1 || ws.seg_last());
+        if (!mbar_wait(full_b + 8 * st, (t / ATT_NST) & 1, abort_word, a.flag) ||
+            !mbar_wait(s_free + 8 * (t & 1), ((t >> 1) & 1) ^ 1, abort_word, a.flag) ||
+            (first && !mbar_wait(q_ready, ks & 1, abort_word, a.flag)))
+          break;
+        tc_fence_after();
+        const uint64_t dt = d_t + (uint64_t)(st * (SM::STAGE / 16));
+        const uint32_t d = tmem + ATT_TM_S + 64 * (t & 1);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_bf16(tmem + ATT_TM_O, dp + 2 * k, dv + 8192 * k / 16, idesc_o, (!first || k > 0) ? 1u : 0u);
-            mma_commit(o_done);
-            mma_commit(empty_b + 8 * st);
-            mma_commit_cta_mask(x_free_b + 8 * xb, (uint16_t)(1u << peer));   // our buffer xb is the peer's to fill
-            if (last) { mma_commit(o_seg); ++ko; }
-            wo.next();
-            ++next_o;
-            did = true;
-          }
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ts(d, tmem + ATT_TM_Q + 32 * j + 8 * k, dt + (j * 1024 + 32 * k) / 16, idesc_s,
+                        (j > 0 || k > 0) ? 1u : 0u);
+        if ((t & 1) == (int)r) {
+          const int ri = (t >> 1) % ATT_NRP;
+          const uint64_t dr = d_rope + (uint64_t)(ri * (8192 / 16));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) mma_bf16(d, d_qpe + 2 * k, dr + 2 * k, idesc_s, 1u);
+          mma_commit(rope_empty + 8 * ri);
         }
-        if (next_s < N) {
-          const int t = next_s, st = t % ATT_NST;
-          const bool first = (t == 0 || ws.lt == 0), last = (t == N - 1 || ws.seg_last());
-          if (mbar_test(full_b + 8 * st, (t / ATT_NST) & 1) && mbar_test(s_free, (t & 1) ^ 1) &&
-              (!first || mbar_test(q_ready, ks & 1))) {
-            tc_fence_after();
-            const uint64_t dt = d_t + (uint64_t)(st * (SM::STAGE / 16));
-            const uint32_t d = tmem + ATT_TM_S;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ts(d, tmem + ATT_TM_Q + 32 * j + 8 * k, dt + (j * 1024 + 32 * k) / 16, idesc_s,
-                            (j > 0 || k > 0) ? 1u : 0u);
-            if ((t & 1) == (int)r) {
-              const uint64_t dr = d_rope + (uint64_t)(st * (SM::STAGE / 16));
-#pragma unroll
-              for (int k = 0; k < 4; ++k) mma_bf16_ts(d, tmem + ATT_TM_QPE + 8 * k, dr + 2 * k, idesc_s, 1u);
-            }
-            mma_commit(s_full);
-            if (last) ++ks;
-            ws.next();
-            ++next_s;
-            did = true;
-          }
-        }
-        if (did) {
-          t_last = global_timer_ns();
-        } else if (*abort_word) {
-          ok = false;
-        } else if (global_timer_ns() - t_last > WAIT_LIMIT_NS) {
-          *abort_word = 1;
-          set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT);
-          ok = false;
-        } else {
-          __nanosleep(32);   // leave the issue slots to the softmax warps on this sub-partition
-        }
+        mma_commit(s_full + 8 * (t & 1));
+        if (last) ++ks;
       }
       mma_commit(fin);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(fin, 0))
         if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
     }
-  } else if (warp >= 10) {
+  } else if (warp == 14) {
+    // ---------------- P.V issuer: O += P(u) . V(u) as soon as P(u) is written ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_bf16(128, 256, 1);
+      const uint64_t d_v = sdesc_sw128_mn_sbo(tile_s, 1024, 4096), d_p = sdesc_sw128(x_s);
+      TileWalk wo{pref, a.n, 0, 0};
+      wo.start(g0);
+      int ko = 0;
+      for (int u = 0; u < N; ++u, wo.next()) {
+        const int st = u % ATT_NST, xb = u & 1;
+        const bool first = (u == 0 || wo.lt == 0), last = (u == N - 1 || wo.seg_last());
+        if (!mbar_wait(p_full_b + 8 * xb, (u >> 1) & 1, abort_word, a.flag) ||
+            (first && ko > 0 && !mbar_wait(o_free, (ko - 1) & 1, abort_word, a.flag)))
+          break;
+        tc_fence_after();
+        const uint64_t dv = d_v + (uint64_t)(st * (SM::STAGE / 16));
+        const uint64_t dp = d_p + (uint64_t)(xb * (16384 / 16));
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(tmem + ATT_TM_O, dp + 2 * k, dv + 8192 * k / 16, idesc_o, (!first || k > 0) ? 1u : 0u);
+        mma_commit(o_done);
+        mma_commit(empty_b + 8 * st);
+        mma_commit_cta_mask(x_free_b + 8 * xb, (uint16_t)(1u << peer));   // our buffer xb is the peer's to fill
+        if (last) { mma_commit(o_seg); ++ko; }
+      }
+      mma_commit(fin);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(fin, 0))
+        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) { set_flag(a.flag, MLA_FLAG_WAIT_TIMEOUT); break; }
+    }
+  } else if (warp >= 10) {   // warps 10-13
     // ---------------- senders: S_r(i) -> staging -> per warp, one bulk copy of its 32 rows into the
     // peer's X, landing on that quarter's barrier (the peer's softmax warps of the quarter wait for it alone)
     const int qs = warp & 3;                              // TMEM lane quarter of this warp
@@ -351,16 +355,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     const uint32_t stg_s = sbase + SM::STG_OFF + 4096 * qs;   // this warp's rows, 4 KB
     uint4* stg_row = (uint4*)(smem + SM::STG_OFF + h * 128);
     for (int i = 0; i < N; ++i) {
-      if (!mbar_wait_warp(s_full, i & 1, abort_word, a.flag)) break;
+      if (!mbar_wait_warp(s_full + 8 * (i & 1), (i >> 1) & 1, abort_word, a.flag)) break;
       tc_fence_after();
       float v[64];
-      const uint32_t sa = tmem + ATT_TM_S + lane_base;
+      const uint32_t sa = tmem + ATT_TM_S + 64 * (i & 1) + lane_base;
 #pragma unroll
       for (int k = 0; k < 4; ++k) tmem_ld16(sa + 16 * k, (uint32_t*)&v[16 * k]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
+      if (lane == 0) mbar_arrive(s_free + 8 * (i & 1));
       if (lane == 0) bulk_wait_read_all();               // this warp's previous copy has left its rows
       __syncwarp();
       // the partial goes out in f16 (half the distributed-shared-memory bytes of fp32; the
@@ -409,14 +413,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         }
         tmem_st16(tmem + ATT_TM_Q + lane_base + 64 * g + 16 * k4, qv);
       }
+      // q_pe row h, chunks 4 g .. 4 g + 3, in the 128-byte-swizzled K-major operand layout
       const uint4* pe = (const uint4*)(a.q_pe + qh * 64 + 32 * g);
-      uint32_t pv[16];
+      uint4* qrow = (uint4*)(smem + SM::QPE_OFF + h * 128);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint4 v = live ? pe[k] : make_uint4(0, 0, 0, 0);
-        pv[4 * k] = v.x; pv[4 * k + 1] = v.y; pv[4 * k + 2] = v.z; pv[4 * k + 3] = v.w;
-      }
-      tmem_st16(tmem + ATT_TM_QPE + lane_base + 16 * g, pv);
+      for (int k = 0; k < 4; ++k) qrow[(4 * g + k) ^ (h & 7)] = live ? pe[k] : make_uint4(0, 0, 0, 0);
+      fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -443,16 +445,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       }
       const int valid = (blk >= 0 && blk < a.n_blocks) ? min(64, seq_len - 64 * lt) : 0;
       if (g == 0 && lane == 0) mbar_arrive_expect_tx(x_full_b + 8 * (4 * xb + q), 4096);   // this quarter's rows
-      if (!mbar_wait_warp(s_full, i & 1, abort_word, a.flag)) { ok = false; break; }
+      if (!mbar_wait_warp(s_full + 8 * xb, (i >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       tc_fence_after();
       float v[32];
-      const uint32_t sp_addr = tmem + ATT_TM_S + 32 * g + lane_base;
+      const uint32_t sp_addr = tmem + ATT_TM_S + 64 * xb + 32 * g + lane_base;
       tmem_ld16(sp_addr, (uint32_t*)&v[0]);
       tmem_ld16(sp_addr + 16, (uint32_t*)&v[16]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);   // the next S may overwrite the buffer
+      if (lane == 0) mbar_arrive(s_free + 8 * xb);   // S(i + 2) may overwrite the buffer
       if (!mbar_wait_warp(x_full_b + 8 * (4 * xb + q), (i >> 1) & 1, abort_word, a.flag)) { ok = false; break; }
       // row h, chunks 4 g .. 4 g + 3 of the peer's partial; P(i) later goes to exactly these bytes
       uint4* xrow = (uint4*)(smem + SM::X_OFF + xb * 16384 + h * 128);
