@@ -28,7 +28,7 @@
 // Every cache byte is read from HBM once and O (128 x 512 fp32) is split over
 // the two CTAs' TMEM. A tile's latent stage is held from its load until its
 // P.V, its rotary block (every other tile) only until its S, so the latent
-// blocks have a 4-deep ring and the rotary blocks 2 slots of their own. S
+// blocks have a 4-deep ring and the rotary blocks 3 slots of their own. S
 // alternates between two TMEM buffers, so S(i + 1) runs, and its partial
 // crosses to the peer, while the softmax still works on S(i). Warps 0-7 run
 // the softmax (warp w: TMEM lane quarter w % 4, column half w / 4), warp 8
@@ -66,7 +66,7 @@ struct TcAttnArgs {
 };
 
 constexpr int ATT_NST = 4;                      // latent ring depth
-constexpr int ATT_NRP = 2;                      // rotary slots (the tiles of this CTA's parity)
+constexpr int ATT_NRP = 3;                      // rotary slots (the tiles of this CTA's parity)
 constexpr int ATT_THREADS = 480;                // 8 softmax, 1 TMA, 1 S-MMA, 4 sender, 1 P.V-MMA warps
 constexpr int ATT_MAX_SEQ = 256;                // sequences per call (the prefix table in shared memory)
 struct AttnSmem {
