@@ -4,6 +4,7 @@
 // run in the GEMM epilogues or in one per-token front-fold kernel.
 #pragma once
 
+#include <atomic>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
@@ -17,6 +18,18 @@
 
 namespace mla {
 namespace tc {
+
+// Raises a kernel's dynamic shared memory limit once per device. The flags are
+// atomic, so host threads launching at the same time are safe; two of them may
+// both make the (idempotent) call. Devices past the table set it on every call.
+template <typename K>
+static void set_smem_once(std::atomic<bool>* done, K kernel, int bytes) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && done[dev].load(std::memory_order_acquire)) return;
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (dev < 64) done[dev].store(true, std::memory_order_release);
+}
 
 // ---------------------------------------------------------------------------
 // TMA tensor maps (cuTensorMapEncodeTiled, resolved through the runtime so the
@@ -104,13 +117,8 @@ template <int BN>
 static int launch_gemm_bn(const CUtensorMap& A, const CUtensorMap& B, const GemmArgs& g, int num_sms,
                           cudaStream_t s) {
   using C = GemmCfg<BN>;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaFuncSetAttribute(tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  set_smem_once(attr_set, tc_gemm_kernel<BN>, C::SMEM);
   const int grid = g.total_units < num_sms ? g.total_units : num_sms;
   launch_pdl(tc_gemm_kernel<BN>, grid, 192, C::SMEM, s, A, B, g);
   mla_count_launch(1);
@@ -150,13 +158,8 @@ template <int BN>
 static int launch_gemm_fp8_bn(const CUtensorMap& A, const CUtensorMap& B, const Fp8GemmArgs& fa, int num_sms,
                               cudaStream_t s) {
   using C = Fp8Cfg<BN>;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaFuncSetAttribute(tc_gemm_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  set_smem_once(attr_set, tc_gemm_fp8_kernel<BN>, C::SMEM);
   const int grid = fa.g.total_units < num_sms ? fa.g.total_units : num_sms;
   launch_pdl(tc_gemm_fp8_kernel<BN>, grid, FP8_THREADS, C::SMEM, s, A, B, fa);
   mla_count_launch(1);
@@ -735,23 +738,13 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     ta.part_o = part_o; ta.part_ml = part_ml; ta.flag = flag;
     ta.ml_r = ml_r = (long long)n * sp * H * 2;   // CTA r's (m, l) copy, one per latent half
     half_cols = 256;
-    static bool attr16[64] = {false}, attr32[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
+    static std::atomic<bool> attr16[64], attr32[64];
     mla_timer_begin("attn", s);
     if (NH == 16) {
-      if (dev < 64 && !attr16[dev]) {
-        cudaFuncSetAttribute(tc_attn_pair_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnPairSmem<16>::SIZE);
-        attr16[dev] = true;
-      }
+      set_smem_once(attr16, tc_attn_pair_kernel<16>, AttnPairSmem<16>::SIZE);
       launch_pdl(tc_attn_pair_kernel<16>, 2 * n * sp, 224, AttnPairSmem<16>::SIZE, s, mqa, mqp, mc, ml, ta);
     } else {
-      if (dev < 64 && !attr32[dev]) {
-        cudaFuncSetAttribute(tc_attn_pair_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnPairSmem<32>::SIZE);
-        attr32[dev] = true;
-      }
+      set_smem_once(attr32, tc_attn_pair_kernel<32>, AttnPairSmem<32>::SIZE);
       launch_pdl(tc_attn_pair_kernel<32>, 2 * n * sp, 224, AttnPairSmem<32>::SIZE, s, mqa, mqp, mc, ml, ta);
     }
     mla_timer_end("attn", s);
@@ -779,13 +772,8 @@ static inline int tc_attention_core(const mla_handle* h, const void* q_abs, cons
     ta.nseg = nseg;
     half_cols = 256;
     seg_counts = nseg;
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr[dev]) {
-      cudaFuncSetAttribute(tc_attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::SIZE);
-      attr[dev] = true;
-    }
+    static std::atomic<bool> attr[64];
+    set_smem_once(attr, tc_attn_decode_kernel, AttnSmem::SIZE);
     mla_timer_begin("attn", s);
     launch_pdl(tc_attn_decode_kernel, 2 * pairs, ATT_THREADS, AttnSmem::SIZE, s, mc, ml, ta);
     mla_timer_end("attn", s);
@@ -1003,13 +991,8 @@ static inline int tc_prefill(const mla_handle* h, const void* hidden, int S, con
     pa.scale_log2 = h->scale * 1.4426950408889634f;
     pa.out = (bf16*)head; pa.flag = flag;
     pa.sink = h->has_sink ? (const float*)(h->base + L.sink) : nullptr;
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr[dev]) {
-      cudaFuncSetAttribute(tc_prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PaSmem::SIZE);
-      attr[dev] = true;
-    }
+    static std::atomic<bool> attr[64];
+    set_smem_once(attr, tc_prefill_attn_kernel, PaSmem::SIZE);
     mla_timer_begin("prefill_attn", s);
     launch_pdl(tc_prefill_attn_kernel, pa.q_tiles * H, 320, PaSmem::SIZE, s, mq, mkv, mkpe, pa);
     mla_timer_end("prefill_attn", s);
