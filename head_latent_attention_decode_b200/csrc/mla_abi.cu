@@ -51,7 +51,7 @@ static int validate_config(const mla_config* c) {
   } else if (c->weight_dtype != c->act_dtype) {
     return MLA_ERR_UNSUPPORTED;
   }
-  // this build's limits
+  // the library's limits
   const long long Hq = (long long)c->n_heads * (c->qk_nope + c->qk_rope);
   if (c->kv_lora_rank % 32 || c->kv_lora_rank > 512) return MLA_ERR_UNSUPPORTED;
   if (c->v_dim % 32 || c->v_dim > 128) return MLA_ERR_UNSUPPORTED;
@@ -279,7 +279,7 @@ const char* mla_strerror(int s) {
   switch (s) {
     case MLA_OK: return "ok";
     case MLA_ERR_INVALID_ARG: return "invalid argument";
-    case MLA_ERR_UNSUPPORTED: return "unsupported by this build";
+    case MLA_ERR_UNSUPPORTED: return "unsupported by this library";
     case MLA_ERR_CUDA: return "CUDA error";
     case MLA_ERR_DEVICE_FLAG: return "device flag set (bad slot, block id or context length)";
     case MLA_ERR_WORKSPACE: return "buffer too small";

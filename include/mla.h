@@ -40,7 +40,7 @@ extern "C" {
 /* ---- status codes ------------------------------------------------------ */
 #define MLA_OK 0
 #define MLA_ERR_INVALID_ARG (-1)   /* bad pointer, size, shape or enum value */
-#define MLA_ERR_UNSUPPORTED (-2)   /* valid request this build does not implement */
+#define MLA_ERR_UNSUPPORTED (-2)   /* valid request this library does not implement */
 #define MLA_ERR_CUDA (-3)          /* a CUDA runtime call or launch failed */
 #define MLA_ERR_DEVICE_FLAG (-4)   /* the device flag is non-zero (see below) */
 #define MLA_ERR_WORKSPACE (-5)     /* workspace / weights buffer too small */
@@ -73,7 +73,7 @@ typedef enum {
 } mla_row_layout;
 
 /* Layer shape ("struct Mla" fields; "MLA Decode QKV Kernel API Reference",
- * Dimensions). Limits of this build: d_r even; r_kv, d_n, d_v, d_r, D and
+ * Dimensions). Limits of this library: d_r even; r_kv, d_n, d_v, d_r, D and
  * H*(d_n+d_r) multiples of 8 (16-byte rows); for MLA_FP8_E4M3_B128 also
  * r_q, d_n, d_v, H*(d_n+d_r) multiples of 128. */
 typedef struct {
